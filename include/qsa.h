@@ -1,0 +1,178 @@
+/*
+ * qsa.h -- C ABI of libqsa.so, the B200 (sm_100a) hot path of Qwen Sparse
+ * Attention (QSA): indexer scores -> exact Top-K over 4-token groups ->
+ * expansion to token ids -> GQA attention over only those tokens of a paged
+ * KV cache.
+ *
+ * The method: "Qwen3.8-27B QSA - BF16 source weights" model card, section
+ * "QSA in brief" (a learned compressed indexer picks 4-token blocks; a fixed
+ * budget plus the current block; all KV stays resident); TensorRT-LLM
+ * "QSASparseAttentionConfig" (exact radix Top-K over compressed groups,
+ * selections expanded to individual tokens, MTP index sharing); "QSA
+ * HiSparse" README (page size 64, FP8 E4M3 KV); the Ascend CANN prefill
+ * article "Qwen4-Exp QSA kommt zu Huaweis Ascend", section "Was der Pull
+ * Request tatsächlich hinzufügt" (-1 padding, zero output for empty rows,
+ * default and explicit softmax scale).
+ *
+ * Conventions shared by every call
+ *  - Memory: every pointer argument is device memory owned by the caller,
+ *    aligned to 16 bytes.  The library never allocates or frees.  Calls that
+ *    need scratch take a caller-provided workspace and report its size
+ *    through a matching *_workspace_size query (a pure host function).
+ *  - Streams: every call only enqueues kernels on `stream` (a cudaStream_t;
+ *    NULL is the legacy default stream) and never synchronises with the host.
+ *  - Errors: argument errors (shapes, dtypes, alignment, workspace size) are
+ *    detected on the host and returned before anything is launched; the
+ *    message is available from qsa_last_error_string() on the calling
+ *    thread.  A launch failure returns QSA_ERR_CUDA.
+ *  - Bad data on the device (a page id outside [0, num_pages), a token id
+ *    outside the page table, a selected group outside the candidates) is
+ *    skipped and ORed into *dev_status as a QSA_DEV_* bit when dev_status is
+ *    not NULL.  No kernel traps.  The status word is only ever ORed into;
+ *    the caller clears it.
+ *  - Layouts (row-major, innermost last):
+ *      indexer query    q_idx        [T, H_I, D_I]          f32 | bf16
+ *      indexer weights  w_idx        [T, H_I]               f32
+ *      indexer keys     k_idx_pages  [num_pages, 16, D_I]   f32 | bf16
+ *                       (one compressed key per 4-token group; a 64-token
+ *                        page holds 16 groups and shares the KV page table)
+ *      KV cache         k_pages, v_pages [num_pages, 64, Hkv, D]
+ *                                                           f32 | bf16 | fp8 e4m3
+ *      page table       page_table   [pt_rows, pt_stride]   int32 physical page ids
+ *      query            q            [T, Hq, D]             f32 | bf16
+ *      output           out          [T, Hq, D]             f32 | bf16
+ *      log-sum-exp      lse          [T, Hq]                f32 (natural log)
+ *    Query token t belongs to request q_req[t] (q_req NULL: request t), a row
+ *    of the page table (a request id outside [0, pt_rows) skips the row and
+ *    sets QSA_DEV_BAD_REQUEST), and sits at absolute position q_pos[t]; its
+ *    current block is group c = q_pos[t] / 4 and its candidates are the
+ *    complete groups 0..c-1.
+ */
+#ifndef QSA_H
+#define QSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define QSA_API __attribute__((visibility("default")))
+#else
+#define QSA_API
+#endif
+
+typedef struct CUstream_st* qsa_stream_t; /* the same type as cudaStream_t */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARG = 1, /* a null pointer, bad shape, misalignment */
+  QSA_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement */
+  QSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+  QSA_ERR_CUDA = 4         /* a CUDA launch or attribute call failed */
+} qsa_status_t;
+
+typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
+
+/* bits ORed into *dev_status by the kernels */
+#define QSA_DEV_BAD_PAGE 1u   /* a page-table entry outside [0, num_pages) */
+#define QSA_DEV_BAD_TOKEN 2u  /* a token id < -1 or beyond the page table */
+#define QSA_DEV_BAD_GROUP 4u  /* a selected group outside the candidates */
+#define QSA_DEV_ROW_RANGE 8u  /* a row's candidates exceed score_stride or
+                                 its tokens exceed W */
+#define QSA_DEV_BAD_REQUEST 16u /* a request id outside [0, pt_rows) */
+
+/* Stage 1 -- indexer scores.
+ * For every query token t and complete group g < c = q_pos[t]/4 (capped at
+ * score_stride):  scores[t*score_stride + g] = sum_h w_idx[t,h] *
+ * ReLU(q_idx[t,h,:] . khat[g,:]), computed in FP32.  khat[g] is row g%16 of
+ * page page_table[q_req[t]][g/16].  Entries g >= c are not written.  A group
+ * whose page id is out of range scores -inf and sets QSA_DEV_BAD_PAGE.
+ * Supported: H_I in {2, 4}, D_I in {32, 64, 128}, q_dt and k_dt F32 or BF16.
+ * The score formula is the one this library fixes for the learned compressed
+ * indexer ("QSA in brief" names the indexer, not its formula). */
+QSA_API qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
+                              const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
+                              const int32_t* page_table, int pt_rows, int pt_stride,
+                              const int32_t* q_req, const int32_t* q_pos, int T, int H_I,
+                              int D_I, float* scores, int score_stride, uint32_t* dev_status,
+                              qsa_stream_t stream);
+
+/* Stage 2 -- exact Top-K over compressed groups (TensorRT-LLM
+ * "QSASparseAttentionConfig", enable_heuristic_topk: the exact radix Top-K).
+ * For every row t, keeps n = min(K, c) of the candidates 0..c-1 (c =
+ * q_pos[t]/4, capped at score_stride) ranked by score descending, ties to the
+ * lower group id (-0.0 ranks equal to +0.0; scores must not be NaN).
+ * sel [T, K] receives the kept group ids in ascending order followed by -1;
+ * n_sel [T] receives n.  c <= K keeps every candidate (dense fallback).
+ * workspace: qsa_topk_groups_workspace_size() bytes (may be 0 / NULL). */
+QSA_API size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride);
+QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, const int32_t* q_pos,
+                             int T, int K, int32_t* sel, int32_t* n_sel, void* workspace,
+                             size_t workspace_bytes, uint32_t* dev_status,
+                             qsa_stream_t stream);
+
+/* Stage 3 -- expansion of the kept groups to token ids ("QSA in brief": the
+ * budget plus the current block; TensorRT-LLM get_indices_block_size: the
+ * selections address single tokens; the MTP index-sharing field).
+ * Row t of tok [T, W] becomes: tokens 4g..4g+3 of each sel[t, 0..n_sel)
+ * entry, then -- when capture_pos is not NULL and p0 = capture_pos[t] <
+ * q_pos[t] -- the groups c(p0)..c(p)-1 completed since the capture, then the
+ * current block 4c(p)..p, then -1 padding.  n_tok[t] = the used width.  A
+ * sel entry outside [0, c(p0)) becomes four -1 slots and sets
+ * QSA_DEV_BAD_GROUP; a row wider than W is cut at W and sets
+ * QSA_DEV_ROW_RANGE.  W >= 4*K + 4 (+4 per group completed since capture). */
+QSA_API qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K,
+                               const int32_t* q_pos, const int32_t* capture_pos, int T,
+                               int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
+                               qsa_stream_t stream);
+
+/* Stage 4 -- GQA attention over the selected tokens ("QSA in brief": only the
+ * selected entries are read; the Ascend article: rows with nothing to attend
+ * give exact zeros, the D-based scale is the default).
+ * For query t and head h (KV head kv = h / (Hq/Hkv)), over the entries j of
+ * tok[t, 0..n_tok[t]) other than -1:
+ *   logit_j = scale * q[t,h,:] . K(j),  out[t,h,:] = sum_j softmax(logit)_j V(j),
+ *   lse[t,h] = log sum_j exp(logit_j)   (-inf and out = 0 for an empty row)
+ * K(j) / V(j) are row (page_table[r][j/64], j%64, kv) of k_pages / v_pages
+ * with r = q_req[t]; FP8 values are code * k_scale (or v_scale); the scales
+ * are ignored for F32 / BF16 caches.  scale = sm_scale, or 1/sqrt(D) when
+ * sm_scale <= 0.  lse may be NULL.
+ * Supported: D in {64, 128, 256}, Hq/Hkv <= 16, q_dt F32 or BF16, kv_dt F32,
+ * BF16 or FP8_E4M3, out_dt F32 or BF16.
+ * _decode splits every row's tokens across CTAs (split-K) and needs
+ * qsa_sparse_attn_decode_workspace_size() bytes of workspace; _prefill
+ * gives each (query, KV head) its own CTA and needs no workspace. */
+QSA_API size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W);
+QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                    const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
+                                    float v_scale, int num_pages, const int32_t* page_table,
+                                    int pt_rows, int pt_stride, const int32_t* q_req,
+                                    const int32_t* tok,
+                                    const int32_t* n_tok, int W, int T, int Hq, int Hkv, int D,
+                                    float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+                                    void* workspace, size_t workspace_bytes,
+                                    uint32_t* dev_status, qsa_stream_t stream);
+
+QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                     const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
+                                     float v_scale, int num_pages, const int32_t* page_table,
+                                     int pt_rows, int pt_stride, const int32_t* q_req,
+                                     const int32_t* tok,
+                                     const int32_t* n_tok, int W, int T, int Hq, int Hkv, int D,
+                                     float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+                                     uint32_t* dev_status, qsa_stream_t stream);
+
+/* Human-readable message for the last non-OK status returned on this thread. */
+QSA_API const char* qsa_last_error_string(void);
+/* Static name of a status code. */
+QSA_API const char* qsa_status_name(qsa_status_t s);
+/* ABI version: bumped on any signature change. */
+QSA_API int qsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QSA_H */

@@ -1,0 +1,154 @@
+// index_scores.cu -- stage 1 of QSA: the indexer score of every complete
+// 4-token group against the query token ("Qwen3.8-27B QSA - BF16 source
+// weights", section "QSA in brief": a learned compressed indexer scores the
+// context in four-token blocks).  Score fixed by this library:
+//   s[t,g] = sum_h w[t,h] * ReLU(q_I[t,h,:] . khat[g,:])      (FP32)
+//
+// Decode-shaped kernel (few query tokens, long context): the pass is bound by
+// HBM reads of the compressed keys (512 B per group at D_I = 128 FP32 against
+// 2 FLOP per byte).  One warp owns one 64-token page at a time = 16 groups x
+// D_I contiguous values (8 KiB at D_I = 128): lane l loads the 16-byte slice
+// [4l, 4l+4) of every group row (16 fully coalesced 512-byte warp loads),
+// accumulates the 16 x H_I partial dots of its slice, and a 5-step butterfly
+// reduce-scatter leaves lane l holding the finished dots of group l/2 for
+// H_I/2 heads; one more shuffle adds the head pair.  Shuffles per group:
+// ~H_I, against 5*H_I for a plain per-group warp reduction.
+#include "qsa_internal.cuh"
+
+namespace qsa {
+namespace {
+
+// One butterfly step of a warp reduce-scatter: lanes with `upper` set keep
+// the upper half of the N-pair window, the others the lower half, and each
+// adds the half its partner (lane ^ mask) gave away.
+template <int N>
+__device__ __forceinline__ void rs_step(float* v, bool upper, int mask) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const float send = upper ? v[i] : v[i + N];
+    const float keep = upper ? v[i + N] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, mask);
+  }
+}
+
+// After this, v[j] for j < V/32 holds the warp-wide sum of value index
+// (V/32)*lane + j.
+template <int V>
+__device__ __forceinline__ void warp_reduce_scatter(float* v, int lane) {
+  static_assert(V >= 32 && (V & (V - 1)) == 0, "V must be a power of two >= 32");
+  rs_step<V / 2>(v, lane & 16, 16);
+  rs_step<V / 4>(v, lane & 8, 8);
+  rs_step<V / 8>(v, lane & 4, 4);
+  rs_step<V / 16>(v, lane & 2, 2);
+  rs_step<V / 32>(v, lane & 1, 1);
+}
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+template <int H_I, int D_I, typename QT, typename KT>
+__global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int warps_per_row) {
+  constexpr int VEC = D_I / 32;          // dims per lane
+  constexpr int V = kPageGroups * H_I;   // partial dots per lane per page
+  constexpr int R = V / 32;              // finished dots per lane (= H_I / 2)
+  const int t = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const int p = a.q_pos[t];
+  int c = p >= 0 ? p / kGroupTokens : 0;
+  if (c > a.score_stride) {
+    if (wid == 0 && lane == 0) flag(a.status, QSA_DEV_ROW_RANGE);
+    c = a.score_stride;
+  }
+  const int npages = (c + kPageGroups - 1) / kPageGroups;
+  if (wid >= npages) return;
+  const int r = a.q_req ? a.q_req[t] : t;
+  const bool bad_req = r < 0 || r >= a.pt_rows;  // every group of the row is skipped
+
+  // this lane's slice of every indexer head of the query
+  float q[H_I][VEC];
+  const QT* qp = reinterpret_cast<const QT*>(a.q_idx) + (size_t)t * H_I * D_I + lane * VEC;
+#pragma unroll
+  for (int h = 0; h < H_I; ++h) VecLoad<QT, VEC>::get(qp, (size_t)h * D_I, q[h]);
+  // weights of the heads whose dots this lane finishes: h = (lane & 1) * R + j
+  float w[R];
+#pragma unroll
+  for (int j = 0; j < R; ++j) w[j] = __ldg(a.w_idx + (size_t)t * H_I + (lane & 1) * R + j);
+
+  const KT* kbase = reinterpret_cast<const KT*>(a.k_idx_pages);
+  const int32_t* pt = a.page_table + (size_t)(bad_req ? 0 : r) * a.pt_stride;
+  float* srow = a.scores + (size_t)t * a.score_stride;
+
+  for (int lp = wid; lp < npages; lp += warps_per_row) {
+    const int g = lp * kPageGroups + (lane >> 1);
+    const int page = (!bad_req && lp < a.pt_stride) ? __ldg(pt + lp) : -1;
+    if (page < 0 || page >= a.num_pages) {  // warp-uniform
+      if (lane == 0) flag(a.status, bad_req ? QSA_DEV_BAD_REQUEST : QSA_DEV_BAD_PAGE);
+      if ((lane & 1) == 0 && g < c) srow[g] = -INFINITY;
+      continue;
+    }
+    const KT* kp = kbase + (size_t)page * kPageGroups * D_I + lane * VEC;
+    float k[kPageGroups][VEC];
+#pragma unroll
+    for (int gi = 0; gi < kPageGroups; ++gi) VecLoad<KT, VEC>::get(kp, (size_t)gi * D_I, k[gi]);
+    float acc[V];
+#pragma unroll
+    for (int gi = 0; gi < kPageGroups; ++gi) {
+#pragma unroll
+      for (int h = 0; h < H_I; ++h) {
+        float d = q[h][0] * k[gi][0];
+#pragma unroll
+        for (int j = 1; j < VEC; ++j) d = fmaf(q[h][j], k[gi][j], d);
+        acc[gi * H_I + h] = d;
+      }
+    }
+    warp_reduce_scatter<V>(acc, lane);
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < R; ++j) s = fmaf(w[j], fmaxf(acc[j], 0.f), s);
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    if ((lane & 1) == 0 && g < c) srow[g] = s;
+  }
+}
+
+template <int H_I, int D_I, typename QT, typename KT>
+cudaError_t launch_typed(const IndexArgs& a, cudaStream_t s) {
+  int cmax = a.score_stride;
+  if (cmax > a.pt_stride * kPageGroups) cmax = a.pt_stride * kPageGroups;
+  const int npages = (cmax + kPageGroups - 1) / kPageGroups;
+  // aim for ~8 resident CTAs of 8 warps on each of the 148 SMs
+  const int target_warps = 148 * 8 * kWarps;
+  int warps_per_row = (target_warps + a.T - 1) / a.T;
+  if (warps_per_row > npages) warps_per_row = npages;
+  if (warps_per_row < 1) warps_per_row = 1;
+  const int blocks = (warps_per_row + kWarps - 1) / kWarps;
+  warps_per_row = blocks * kWarps;
+  dim3 grid(blocks, a.T);
+  index_scores_kernel<H_I, D_I, QT, KT><<<grid, kThreads, 0, s>>>(a, warps_per_row);
+  return cudaGetLastError();
+}
+
+template <int H_I, int D_I>
+cudaError_t launch_dims(const IndexArgs& a, cudaStream_t s) {
+  if (a.q_dt == QSA_F32 && a.k_dt == QSA_F32) return launch_typed<H_I, D_I, float, float>(a, s);
+  if (a.q_dt == QSA_F32 && a.k_dt == QSA_BF16) return launch_typed<H_I, D_I, float, __nv_bfloat16>(a, s);
+  if (a.q_dt == QSA_BF16 && a.k_dt == QSA_F32) return launch_typed<H_I, D_I, __nv_bfloat16, float>(a, s);
+  return launch_typed<H_I, D_I, __nv_bfloat16, __nv_bfloat16>(a, s);
+}
+
+}  // namespace
+
+cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t s) {
+  if (a.T == 0) return cudaSuccess;
+  switch (a.H_I * 1000 + a.D_I) {
+    case 2032: return launch_dims<2, 32>(a, s);
+    case 2064: return launch_dims<2, 64>(a, s);
+    case 2128: return launch_dims<2, 128>(a, s);
+    case 4032: return launch_dims<4, 32>(a, s);
+    case 4064: return launch_dims<4, 64>(a, s);
+    case 4128: return launch_dims<4, 128>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qsa

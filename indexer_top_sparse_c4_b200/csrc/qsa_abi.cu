@@ -1,0 +1,190 @@
+// qsa_abi.cu -- the extern "C" entry points of libqsa.so (include/qsa.h):
+// host-side argument validation, then one launch per stage on the caller's
+// stream.  No allocation, no host synchronisation.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "qsa_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+qsa_status_t fail(qsa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+qsa_status_t cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return QSA_OK;
+  return fail(QSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+#define REQUIRE(cond, ...) \
+  do {                     \
+    if (!(cond)) return fail(QSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+#define SUPPORT(cond, ...) \
+  do {                     \
+    if (!(cond)) return fail(QSA_ERR_UNSUPPORTED, __VA_ARGS__); \
+  } while (0)
+
+constexpr int kMaxGridY = 65535;
+
+qsa_status_t check_attn(const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages,
+                        qsa_dtype_t kv_dt, int num_pages, const int32_t* page_table, int pt_rows,
+                        int pt_stride,
+                        const int32_t* tok, const int32_t* n_tok, int W, int T, int Hq, int Hkv,
+                        int D, void* out, qsa_dtype_t out_dt, float k_scale, float v_scale) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  REQUIRE(Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0, "need Hq %% Hkv == 0 (Hq=%d, Hkv=%d)", Hq, Hkv);
+  SUPPORT(Hq / Hkv <= 16, "at most 16 query heads per KV head (got %d)", Hq / Hkv);
+  SUPPORT(D == 64 || D == 128 || D == 256, "head dim D must be 64, 128 or 256 (got %d)", D);
+  REQUIRE(W >= 1, "W must be >= 1 (got %d)", W);
+  REQUIRE(num_pages >= 1 && pt_rows >= 1 && pt_stride >= 1,
+          "num_pages, pt_rows and pt_stride must be >= 1");
+  REQUIRE(q_dt == QSA_F32 || q_dt == QSA_BF16, "q dtype must be F32 or BF16");
+  REQUIRE(kv_dt == QSA_F32 || kv_dt == QSA_BF16 || kv_dt == QSA_FP8_E4M3, "bad KV dtype");
+  REQUIRE(out_dt == QSA_F32 || out_dt == QSA_BF16, "out dtype must be F32 or BF16");
+  if (kv_dt == QSA_FP8_E4M3)
+    REQUIRE(isfinite(k_scale) && isfinite(v_scale) && k_scale > 0.f && v_scale > 0.f,
+            "FP8 scales must be finite and > 0");
+  if (T == 0) return QSA_OK;
+  REQUIRE(q && k_pages && v_pages && page_table && tok && n_tok && out, "null pointer argument");
+  REQUIRE(aligned16(q) && aligned16(k_pages) && aligned16(v_pages) && aligned16(out),
+          "q, k_pages, v_pages and out must be 16-byte aligned");
+  return QSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qsa_last_error_string(void) { return g_err; }
+
+const char* qsa_status_name(qsa_status_t s) {
+  switch (s) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARG: return "QSA_ERR_INVALID_ARG";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+int qsa_abi_version(void) { return 1; }
+
+qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
+                              const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
+                              const int32_t* page_table, int pt_rows, int pt_stride,
+                              const int32_t* q_req,
+                              const int32_t* q_pos, int T, int H_I, int D_I, float* scores,
+                              int score_stride, uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  SUPPORT((H_I == 2 || H_I == 4) && (D_I == 32 || D_I == 64 || D_I == 128),
+          "indexer shape H_I=%d, D_I=%d not built (H_I in {2,4}, D_I in {32,64,128})", H_I, D_I);
+  REQUIRE(q_dt == QSA_F32 || q_dt == QSA_BF16, "q_idx dtype must be F32 or BF16");
+  REQUIRE(k_dt == QSA_F32 || k_dt == QSA_BF16, "k_idx_pages dtype must be F32 or BF16");
+  REQUIRE(score_stride >= 1 && pt_stride >= 1 && pt_rows >= 1 && num_pages >= 1,
+          "score_stride, pt_rows, pt_stride and num_pages must be >= 1");
+  if (T == 0) return QSA_OK;
+  REQUIRE(q_idx && w_idx && k_idx_pages && page_table && q_pos && scores, "null pointer argument");
+  REQUIRE(aligned16(q_idx) && aligned16(k_idx_pages), "q_idx and k_idx_pages must be 16-byte aligned");
+  qsa::IndexArgs a{q_idx, q_dt, w_idx, k_idx_pages, k_dt, num_pages, page_table, pt_rows, pt_stride,
+                   q_req, q_pos, T, H_I, D_I, scores, score_stride, dev_status};
+  return cuda_status(qsa::launch_index_scores(a, (cudaStream_t)stream), "qsa_index_scores launch");
+}
+
+size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride) {
+  (void)T; (void)K; (void)score_stride;
+  return 0;
+}
+
+qsa_status_t qsa_topk_groups(const float* scores, int score_stride, const int32_t* q_pos, int T,
+                             int K, int32_t* sel, int32_t* n_sel, void* workspace,
+                             size_t workspace_bytes, uint32_t* dev_status, qsa_stream_t stream) {
+  (void)workspace; (void)workspace_bytes;
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
+  REQUIRE(score_stride >= 1, "score_stride must be >= 1");
+  SUPPORT(qsa::topk_cluster_size(score_stride) > 0, "score_stride %d exceeds the %d groups a row may hold",
+          score_stride, 8 * 49152);
+  if (T == 0) return QSA_OK;
+  REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
+  qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
+  return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups launch");
+}
+
+qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos,
+                               const int32_t* capture_pos, int T, int32_t* tok, int32_t* n_tok,
+                               int W, uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
+  REQUIRE(W >= 4 * K + 4, "W must be >= 4*K + 4 = %d (got %d)", 4 * K + 4, W);
+  if (T == 0) return QSA_OK;
+  REQUIRE(sel && n_sel && q_pos && tok && n_tok, "null pointer argument");
+  qsa::ExpandArgs a{sel, n_sel, K, q_pos, capture_pos, T, tok, n_tok, W, dev_status};
+  return cuda_status(qsa::launch_expand_select(a, (cudaStream_t)stream), "qsa_expand_select launch");
+}
+
+size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W) {
+  if (T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return 0;
+  return qsa::attn_decode_ws_bytes(T, Hq, D, qsa::attn_decode_splits(T, Hkv, W));
+}
+
+qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                    const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
+                                    float v_scale, int num_pages, const int32_t* page_table,
+                                    int pt_rows, int pt_stride, const int32_t* q_req,
+                                    const int32_t* tok,
+                                    const int32_t* n_tok, int W, int T, int Hq, int Hkv, int D,
+                                    float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+                                    void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                                    qsa_stream_t stream) {
+  qsa_status_t st = check_attn(q, q_dt, k_pages, v_pages, kv_dt, num_pages, page_table, pt_rows,
+                               pt_stride,
+                               tok, n_tok, W, T, Hq, Hkv, D, out, out_dt, k_scale, v_scale);
+  if (st != QSA_OK || T == 0) return st;
+  const int splits = qsa::attn_decode_splits(T, Hkv, W);
+  const size_t need = qsa::attn_decode_ws_bytes(T, Hq, D, splits);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(QSA_ERR_WORKSPACE, "decode needs %zu bytes of 16-byte-aligned workspace (got %zu)",
+                need, workspace ? workspace_bytes : (size_t)0);
+  qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
+                  pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
+                  dev_status};
+  return cuda_status(qsa::launch_sparse_attn(a, splits, workspace, (cudaStream_t)stream),
+                     "qsa_sparse_attn_decode launch");
+}
+
+qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                     const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
+                                     float v_scale, int num_pages, const int32_t* page_table,
+                                     int pt_rows, int pt_stride, const int32_t* q_req,
+                                     const int32_t* tok,
+                                     const int32_t* n_tok, int W, int T, int Hq, int Hkv, int D,
+                                     float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+                                     uint32_t* dev_status, qsa_stream_t stream) {
+  qsa_status_t st = check_attn(q, q_dt, k_pages, v_pages, kv_dt, num_pages, page_table, pt_rows,
+                               pt_stride,
+                               tok, n_tok, W, T, Hq, Hkv, D, out, out_dt, k_scale, v_scale);
+  if (st != QSA_OK || T == 0) return st;
+  qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
+                  pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
+                  dev_status};
+  return cuda_status(qsa::launch_sparse_attn(a, 1, nullptr, (cudaStream_t)stream),
+                     "qsa_sparse_attn_prefill launch");
+}
+
+}  // extern "C"

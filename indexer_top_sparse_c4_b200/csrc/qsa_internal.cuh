@@ -1,0 +1,146 @@
+// qsa_internal.cuh -- shared device helpers and the internal launcher
+// declarations of libqsa.so.  Not part of the public ABI (include/qsa.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <stdint.h>
+
+#include "../../include/qsa.h"
+
+namespace qsa {
+
+constexpr int kPageTokens = 64;                        // tokens per KV page
+constexpr int kGroupTokens = 4;                        // tokens per compressed group (C4)
+constexpr int kPageGroups = kPageTokens / kGroupTokens;  // groups per page
+
+// ---- value loads ----------------------------------------------------------------
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float get(const float* p, size_t i) { return __ldg(p + i); }
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float get(const __nv_bfloat16* p, size_t i) {
+    return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short*>(p) + i));
+  }
+};
+template <> struct Elem<__nv_fp8_e4m3> {
+  static __device__ __forceinline__ float get(const __nv_fp8_e4m3* p, size_t i) {
+    const __nv_fp8_storage_t c = __ldg(reinterpret_cast<const unsigned char*>(p) + i);
+    return __half2float(__half(__nv_cvt_fp8_to_halfraw(c, __NV_E4M3)));
+  }
+};
+
+// Load N consecutive elements starting at element index i (i*sizeof(T) and
+// N*sizeof(T) chosen by the callers so the access is a single aligned vector
+// load) and widen them to float.
+template <typename T, int N> struct VecLoad;
+template <int N> struct VecLoad<float, N> {
+  static __device__ __forceinline__ void get(const float* p, size_t i, float* out) {
+    if constexpr (N == 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(p + i));
+      out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else if constexpr (N == 2) {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(p + i));
+      out[0] = v.x; out[1] = v.y;
+    } else if constexpr (N == 8) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(p + i));
+      const float4 b = __ldg(reinterpret_cast<const float4*>(p + i + 4));
+      out[0] = a.x; out[1] = a.y; out[2] = a.z; out[3] = a.w;
+      out[4] = b.x; out[5] = b.y; out[6] = b.z; out[7] = b.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) out[j] = __ldg(p + i + j);
+    }
+  }
+};
+template <int N> struct VecLoad<__nv_bfloat16, N> {
+  static __device__ __forceinline__ void get(const __nv_bfloat16* p, size_t i, float* out) {
+    const unsigned short* s = reinterpret_cast<const unsigned short*>(p) + i;
+    if constexpr (N == 8) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(s));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        out[2 * j] = __uint_as_float(w[j] << 16);
+        out[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+      }
+    } else if constexpr (N == 4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(s));
+      out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+      out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+    } else if constexpr (N == 2) {
+      const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(s));
+      out[0] = __uint_as_float(v << 16); out[1] = __uint_as_float(v & 0xffff0000u);
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) out[j] = bf16_bits_to_f32(__ldg(s + j));
+    }
+  }
+};
+template <int N> struct VecLoad<__nv_fp8_e4m3, N> {
+  static __device__ __forceinline__ void get(const __nv_fp8_e4m3* p, size_t i, float* out) {
+    const unsigned char* s = reinterpret_cast<const unsigned char*>(p) + i;
+    if constexpr (N == 8) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(s));
+      const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] & 0xffffu), __NV_E4M3);
+        const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w[j] >> 16), __NV_E4M3);
+        const float2 a = __half22float2(__half2(lo));
+        const float2 b = __half22float2(__half2(hi));
+        out[4 * j] = a.x; out[4 * j + 1] = a.y; out[4 * j + 2] = b.x; out[4 * j + 3] = b.y;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < N; ++j) out[j] = Elem<__nv_fp8_e4m3>::get(p, i + j);
+    }
+  }
+};
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// ---- launchers (one per stage; defined in the stage's .cu file) -----------------
+
+struct IndexArgs {
+  const void* q_idx; qsa_dtype_t q_dt; const float* w_idx;
+  const void* k_idx_pages; qsa_dtype_t k_dt; int num_pages;
+  const int32_t* page_table; int pt_rows, pt_stride; const int32_t* q_req; const int32_t* q_pos;
+  int T, H_I, D_I; float* scores; int score_stride; uint32_t* status;
+};
+cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t s);
+
+struct TopkArgs {
+  const float* scores; int score_stride; const int32_t* q_pos; int T, K;
+  int32_t* sel; int32_t* n_sel; uint32_t* status;
+};
+int topk_cluster_size(int score_stride);       // 0: unsupported
+cudaError_t launch_topk_groups(const TopkArgs& a, cudaStream_t s);
+
+struct ExpandArgs {
+  const int32_t* sel; const int32_t* n_sel; int K; const int32_t* q_pos;
+  const int32_t* capture_pos; int T; int32_t* tok; int32_t* n_tok; int W; uint32_t* status;
+};
+cudaError_t launch_expand_select(const ExpandArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+  const void* q; qsa_dtype_t q_dt; const void* k_pages; const void* v_pages; qsa_dtype_t kv_dt;
+  float k_scale, v_scale; int num_pages; const int32_t* page_table; int pt_rows, pt_stride;
+  const int32_t* q_req; const int32_t* tok; const int32_t* n_tok; int W, T, Hq, Hkv, D;
+  float sm_scale; void* out; qsa_dtype_t out_dt; float* lse; uint32_t* status;
+};
+// splits > 1: partial (o, m, l) per split go to ws_o / ws_ml and a combine
+// kernel finishes; splits == 1 writes out / lse directly.
+int attn_decode_splits(int T, int Hkv, int W);
+size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
+cudaError_t launch_sparse_attn(const AttnArgs& a, int splits, void* ws, cudaStream_t s);
+
+}  // namespace qsa

@@ -1,0 +1,252 @@
+// sparse_attn.cu -- stage 4 of QSA: GQA attention over only the selected
+// tokens of a paged KV cache ("Qwen3.8-27B QSA - BF16 source weights", "QSA in
+// brief": the selection decides which cache entries are read, nothing is
+// compressed; Ascend CANN article, "Was der Pull Request tatsächlich
+// hinzufügt": empty rows produce exact zeros, the 1/sqrt(D) scale is kept).
+//
+// General kernel (every dtype, D in {64,128,256}, up to 16 query heads per KV
+// head).  CTA = (token split, KV head, query token).  Each warp walks every
+// 4th selected token of the split: lane l holds dims [l*D/32, (l+1)*D/32) of
+// the gathered K and V rows (one coalesced vector load each), the per-head
+// dots are finished with a warp all-reduce, and an online softmax in base 2
+// keeps a running max / sum per head with the unnormalised output in shared
+// memory.  The four warps are merged at the end; with several splits the
+// partial (o, max, sum) go to the workspace and a combine kernel finishes.
+#include <math.h>
+
+#include "qsa_internal.cuh"
+
+namespace qsa {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxG = 16;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+struct AttnScales {
+  float qk;    // softmax scale * log2(e) (* k_scale for FP8): logits in base 2
+  float vmul;  // v_scale for FP8, 1 otherwise
+};
+
+template <typename OT> __device__ __forceinline__ void store_out(OT* p, size_t i, float v);
+template <> __device__ __forceinline__ void store_out<float>(float* p, size_t i, float v) { p[i] = v; }
+template <> __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, size_t i, float v) {
+  p[i] = __float2bfloat16_rn(v);
+}
+
+template <int D, typename QT, typename KVT, typename OT>
+__global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, AttnScales sc, int splits,
+                                                             int chunk, float* ws_o, float* ws_ml) {
+  constexpr int VPT = D / 32;
+  extern __shared__ __align__(16) float smem[];
+  const int G = a.Hq / a.Hkv;
+  float* q_s = smem;                        // [G][D]       scaled query
+  float* o_s = q_s + G * D;                 // [warps][G][D] unnormalised outputs
+  float* ml_s = o_s + kWarps * G * D;       // [warps][kMaxG][2] running max / sum
+  const int s = blockIdx.x, kvh = blockIdx.y, t = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h0 = kvh * G;
+
+  const QT* qp = reinterpret_cast<const QT*>(a.q) + ((size_t)t * a.Hq + h0) * D;
+  for (int i = tid; i < G * D; i += kThreads) q_s[i] = Elem<QT>::get(qp, i) * sc.qk;
+  for (int i = tid; i < kWarps * G * D; i += kThreads) o_s[i] = 0.f;
+  __syncthreads();
+
+  float m[kMaxG], l[kMaxG];
+#pragma unroll
+  for (int h = 0; h < kMaxG; ++h) { m[h] = -INFINITY; l[h] = 0.f; }
+
+  int r = a.q_req ? a.q_req[t] : t;
+  int nt = a.n_tok[t];
+  nt = nt < 0 ? 0 : (nt > a.W ? a.W : nt);
+  if (r < 0 || r >= a.pt_rows) {  // the whole row is skipped: zero output
+    if (tid == 0 && s == 0) flag(a.status, QSA_DEV_BAD_REQUEST);
+    r = 0;
+    nt = 0;
+  }
+  const int beg = s * chunk;
+  const int end = nt < beg + chunk ? nt : beg + chunk;
+  const int32_t* trow = a.tok + (size_t)t * a.W;
+  const int32_t* pt = a.page_table + (size_t)r * a.pt_stride;
+  const KVT* kc = reinterpret_cast<const KVT*>(a.k_pages);
+  const KVT* vc = reinterpret_cast<const KVT*>(a.v_pages);
+  float* o_w = o_s + warp * G * D;
+
+  for (int i = beg + warp; i < end; i += kWarps) {
+    const int j = __ldg(trow + i);
+    if (j == -1) continue;
+    if (j < -1 || (j / kPageTokens) >= a.pt_stride) {
+      if (lane == 0) flag(a.status, QSA_DEV_BAD_TOKEN);
+      continue;
+    }
+    const int page = __ldg(pt + j / kPageTokens);
+    if (page < 0 || page >= a.num_pages) {
+      if (lane == 0) flag(a.status, QSA_DEV_BAD_PAGE);
+      continue;
+    }
+    const size_t base = (((size_t)page * kPageTokens + (j % kPageTokens)) * a.Hkv + kvh) * D + lane * VPT;
+    float kf[VPT], vf[VPT];
+    VecLoad<KVT, VPT>::get(kc, base, kf);
+    VecLoad<KVT, VPT>::get(vc, base, vf);
+    float dot[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {
+        const float* qh = q_s + h * D + lane * VPT;
+        float d = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < VPT; ++jj) d = fmaf(qh[jj], kf[jj], d);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        dot[h] = d;
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {
+        const float mn = fmaxf(m[h], dot[h]);
+        const float alpha = exp2f(m[h] - mn);
+        const float pr = exp2f(dot[h] - mn);
+        l[h] = l[h] * alpha + pr;
+        m[h] = mn;
+        float* oh = o_w + h * D + lane * VPT;
+#pragma unroll
+        for (int jj = 0; jj < VPT; ++jj) oh[jj] = fmaf(oh[jj], alpha, pr * vf[jj]);
+      }
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < G) {
+        ml_s[(warp * kMaxG + h) * 2] = m[h];
+        ml_s[(warp * kMaxG + h) * 2 + 1] = l[h];
+      }
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < G * D; idx += kThreads) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, ml_s[(w * kMaxG + h) * 2]);
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = ml_s[(w * kMaxG + h) * 2];
+        if (mw == -INFINITY) continue;
+        const float f = exp2f(mw - M);
+        L = fmaf(ml_s[(w * kMaxG + h) * 2 + 1], f, L);
+        O = fmaf(o_s[(w * G + h) * D + d], f, O);
+      }
+    }
+    const size_t th = (size_t)t * a.Hq + h0 + h;
+    if (splits == 1) {
+      store_out<OT>(reinterpret_cast<OT*>(a.out), th * D + d, L > 0.f ? O / L * sc.vmul : 0.f);
+      if (d == 0 && a.lse) a.lse[th] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    } else {
+      ws_o[(th * splits + s) * D + d] = O;
+      if (d == 0) {
+        ws_ml[(th * splits + s) * 2] = M;
+        ws_ml[(th * splits + s) * 2 + 1] = L;
+      }
+    }
+  }
+}
+
+// Merge the per-split partials of one (query, head): rescale every split to
+// the common maximum, add, normalise.
+template <typename OT>
+__global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs a, AttnScales sc, int splits,
+                                                           const float* ws_o, const float* ws_ml) {
+  const size_t th = blockIdx.x;
+  const float* ml = ws_ml + th * splits * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
+  float L = 0.f;
+  if (M != -INFINITY)
+    for (int s = 0; s < splits; ++s)
+      if (ml[2 * s] != -INFINITY) L = fmaf(ml[2 * s + 1], exp2f(ml[2 * s] - M), L);
+  for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
+    float O = 0.f;
+    if (L > 0.f)
+      for (int s = 0; s < splits; ++s)
+        if (ml[2 * s] != -INFINITY) O = fmaf(ws_o[(th * splits + s) * a.D + d], exp2f(ml[2 * s] - M), O);
+    store_out<OT>(reinterpret_cast<OT*>(a.out), th * a.D + d, L > 0.f ? O / L * sc.vmul : 0.f);
+  }
+  if (threadIdx.x == 0 && a.lse) a.lse[th] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+}
+
+template <int D, typename QT, typename KVT, typename OT>
+cudaError_t launch_typed(const AttnArgs& a, const AttnScales& sc, int splits, void* ws,
+                         cudaStream_t s) {
+  const int G = a.Hq / a.Hkv;
+  const size_t smem = ((size_t)(1 + kWarps) * G * D + kWarps * kMaxG * 2) * sizeof(float);
+  auto kern = attn_simt_kernel<D, QT, KVT, OT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int chunk = (a.W + splits - 1) / splits;
+  float* ws_o = reinterpret_cast<float*>(ws);
+  float* ws_ml = ws_o ? ws_o + (size_t)a.T * a.Hq * splits * D : nullptr;
+  kern<<<dim3(splits, a.Hkv, a.T), kThreads, smem, s>>>(a, sc, splits, chunk, ws_o, ws_ml);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  attn_combine_kernel<OT><<<a.T * a.Hq, D < 256 ? D : 256, 0, s>>>(a, sc, splits, ws_o, ws_ml);
+  return cudaGetLastError();
+}
+
+template <int D, typename QT, typename KVT>
+cudaError_t launch_out(const AttnArgs& a, const AttnScales& sc, int splits, void* ws, cudaStream_t s) {
+  if (a.out_dt == QSA_F32) return launch_typed<D, QT, KVT, float>(a, sc, splits, ws, s);
+  return launch_typed<D, QT, KVT, __nv_bfloat16>(a, sc, splits, ws, s);
+}
+
+template <int D, typename QT>
+cudaError_t launch_kv(const AttnArgs& a, const AttnScales& sc, int splits, void* ws, cudaStream_t s) {
+  switch (a.kv_dt) {
+    case QSA_F32: return launch_out<D, QT, float>(a, sc, splits, ws, s);
+    case QSA_BF16: return launch_out<D, QT, __nv_bfloat16>(a, sc, splits, ws, s);
+    default: return launch_out<D, QT, __nv_fp8_e4m3>(a, sc, splits, ws, s);
+  }
+}
+
+template <int D>
+cudaError_t launch_q(const AttnArgs& a, const AttnScales& sc, int splits, void* ws, cudaStream_t s) {
+  if (a.q_dt == QSA_F32) return launch_kv<D, float>(a, sc, splits, ws, s);
+  return launch_kv<D, __nv_bfloat16>(a, sc, splits, ws, s);
+}
+
+}  // namespace
+
+int attn_decode_splits(int T, int Hkv, int W) {
+  // enough CTAs to cover the 148 SMs several times, at least 32 tokens each
+  const int rows = T * Hkv > 0 ? T * Hkv : 1;
+  int splits = (4 * 148 + rows - 1) / rows;
+  const int max_splits = (W + 31) / 32;
+  if (splits > max_splits) splits = max_splits;
+  return splits < 1 ? 1 : splits;
+}
+
+size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
+  if (splits <= 1) return 0;
+  return (size_t)T * Hq * splits * (D + 2) * sizeof(float);
+}
+
+cudaError_t launch_sparse_attn(const AttnArgs& a, int splits, void* ws, cudaStream_t s) {
+  if (a.T == 0) return cudaSuccess;
+  const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
+  const bool fp8 = a.kv_dt == QSA_FP8_E4M3;
+  AttnScales sc;
+  sc.qk = (float)(scale * 1.4426950408889634 * (fp8 ? (double)a.k_scale : 1.0));
+  sc.vmul = fp8 ? a.v_scale : 1.f;
+  switch (a.D) {
+    case 64: return launch_q<64>(a, sc, splits, ws, s);
+    case 128: return launch_q<128>(a, sc, splits, ws, s);
+    case 256: return launch_q<256>(a, sc, splits, ws, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qsa

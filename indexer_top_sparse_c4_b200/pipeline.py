@@ -1,0 +1,75 @@
+"""One QSA step over a Workload: device buffers (allocated once with torch) and
+the four library calls in order on one stream.
+
+    scores  <- qsa_index_scores      (query position, or the capture position
+                                       when an MTP draft reuses a selection)
+    sel     <- qsa_topk_groups
+    tok     <- qsa_expand_select
+    out     <- qsa_sparse_attn_decode / qsa_sparse_attn_prefill
+
+This is plumbing only: torch provides memory and the stream, libqsa.so does
+all the work.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import qsa
+from .workloads import GROUP_TOKENS, Workload
+
+
+class QSAStep:
+    def __init__(self, w: Workload, prefill: bool | None = None, out_dtype=None):
+        self.w = w
+        dev = w.q.device
+        self.prefill = (w.T > 64) if prefill is None else prefill
+        self.sel_pos = w.capture_pos if w.capture_pos is not None else w.q_pos
+        self.score_stride = max(1, int(self.sel_pos.max().item()) // GROUP_TOKENS)
+        T = w.T
+        self.scores = torch.empty((T, self.score_stride), dtype=torch.float32, device=dev)
+        self.sel = torch.empty((T, w.K), dtype=torch.int32, device=dev)
+        self.n_sel = torch.empty((T,), dtype=torch.int32, device=dev)
+        self.tok = torch.empty((T, w.W), dtype=torch.int32, device=dev)
+        self.n_tok = torch.empty((T,), dtype=torch.int32, device=dev)
+        if out_dtype is None:
+            out_dtype = torch.float32 if w.q.dtype == torch.float32 else torch.bfloat16
+        self.out = torch.empty((T, w.Hq, w.D), dtype=out_dtype, device=dev)
+        self.lse = torch.empty((T, w.Hq), dtype=torch.float32, device=dev)
+        self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
+        ws = 0 if self.prefill else qsa.qsa_sparse_attn_decode_workspace_size(T, w.Hq, w.Hkv, w.D, w.W)
+        self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
+        tk = qsa.qsa_topk_groups_workspace_size(T, w.K, self.score_stride)
+        self.topk_ws = torch.empty((max(tk, 16),), dtype=torch.uint8, device=dev) if tk else None
+
+    # the four stages, separately callable for per-stage tests and timing
+    def index_scores(self, stream=None):
+        w = self.w
+        qsa.qsa_index_scores(w.q_idx, w.w_idx, w.k_idx_pages, w.page_table, self.sel_pos,
+                             self.scores, q_req=w.q_req, dev_status=self.status, stream=stream)
+
+    def topk(self, stream=None):
+        qsa.qsa_topk_groups(self.scores, self.sel_pos, self.w.K, self.sel, self.n_sel,
+                            workspace=self.topk_ws, dev_status=self.status, stream=stream)
+
+    def expand(self, stream=None):
+        w = self.w
+        qsa.qsa_expand_select(self.sel, self.n_sel, w.q_pos, self.tok, self.n_tok,
+                              capture_pos=w.capture_pos, dev_status=self.status, stream=stream)
+
+    def attention(self, stream=None, sm_scale=0.0):
+        w = self.w
+        common = dict(k_scale=w.k_scale, v_scale=w.v_scale, q_req=w.q_req, sm_scale=sm_scale,
+                      lse=self.lse, dev_status=self.status, stream=stream)
+        if self.prefill:
+            qsa.qsa_sparse_attn_prefill(w.q, w.k_pages, w.v_pages, w.page_table, self.tok,
+                                        self.n_tok, self.out, **common)
+        else:
+            qsa.qsa_sparse_attn_decode(w.q, w.k_pages, w.v_pages, w.page_table, self.tok,
+                                       self.n_tok, self.out, workspace=self.ws, **common)
+
+    def run(self, stream=None, sm_scale=0.0):
+        self.index_scores(stream)
+        self.topk(stream)
+        self.expand(stream)
+        self.attention(stream, sm_scale)
+        return self.out

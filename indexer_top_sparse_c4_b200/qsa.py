@@ -1,0 +1,181 @@
+"""Thin ctypes binding of libqsa.so (include/qsa.h).
+
+Same names as the C entry points.  Each function only turns torch tensors
+into pointers, dtypes and sizes and calls the library on the current CUDA
+stream; every step of the computation runs in the library's kernels.  There
+is no fallback: if libqsa.so is missing or a call fails, an exception is
+raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqsa.so")
+
+QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = range(5)
+QSA_F32, QSA_BF16, QSA_FP8_E4M3 = 0, 1, 2
+QSA_DEV_BAD_PAGE, QSA_DEV_BAD_TOKEN, QSA_DEV_BAD_GROUP, QSA_DEV_ROW_RANGE = 1, 2, 4, 8
+QSA_DEV_BAD_REQUEST = 16
+
+ENTRY_POINTS = (
+    "qsa_index_scores", "qsa_topk_groups_workspace_size", "qsa_topk_groups",
+    "qsa_expand_select", "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
+    "qsa_sparse_attn_prefill", "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
+)
+
+
+class QSAError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{_status_name(status)}: {msg}")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqsa.so (built in-tree by ``python -m indexer_top_sparse_c4_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m indexer_top_sparse_c4_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.qsa_index_scores.argtypes = [P, I, P, P, I, I, P, I, I, P, P, I, I, I, P, I, P, P]
+    L.qsa_topk_groups_workspace_size.argtypes = [I, I, I]
+    L.qsa_topk_groups_workspace_size.restype = U
+    L.qsa_topk_groups.argtypes = [P, I, P, I, I, P, P, P, U, P, P]
+    L.qsa_expand_select.argtypes = [P, P, I, P, P, I, P, P, I, P, P]
+    L.qsa_sparse_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
+    L.qsa_sparse_attn_decode_workspace_size.restype = U
+    L.qsa_sparse_attn_decode.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
+                                         F, P, I, P, P, U, P, P]
+    L.qsa_sparse_attn_prefill.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
+                                          F, P, I, P, P, P]
+    for name in ("qsa_index_scores", "qsa_topk_groups", "qsa_expand_select",
+                 "qsa_sparse_attn_decode", "qsa_sparse_attn_prefill"):
+        getattr(L, name).restype = I
+    L.qsa_last_error_string.restype = ctypes.c_char_p
+    L.qsa_status_name.restype = ctypes.c_char_p
+    L.qsa_status_name.argtypes = [I]
+    L.qsa_abi_version.restype = I
+    _lib = L
+    return L
+
+
+def _status_name(s: int) -> str:
+    try:
+        return lib().qsa_status_name(s).decode()
+    except Exception:
+        return f"status {s}"
+
+
+def _check(status: int):
+    if status != QSA_OK:
+        raise QSAError(status, lib().qsa_last_error_string().decode())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("libqsa takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return QSA_F32
+    if t.dtype == torch.bfloat16:
+        return QSA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return QSA_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def qsa_index_scores(q_idx, w_idx, k_idx_pages, page_table, q_pos, scores, q_req=None,
+                     dev_status=None, stream=None):
+    T, H_I, D_I = q_idx.shape
+    _check(lib().qsa_index_scores(
+        _ptr(q_idx), _dt(q_idx), _ptr(w_idx), _ptr(k_idx_pages), _dt(k_idx_pages),
+        k_idx_pages.shape[0], _ptr(page_table), page_table.shape[0], page_table.shape[1],
+        _ptr(q_req), _ptr(q_pos),
+        T, H_I, D_I, _ptr(scores), scores.shape[1], _ptr(dev_status), _stream(stream)))
+    return scores
+
+
+def qsa_topk_groups_workspace_size(T, K, score_stride) -> int:
+    return int(lib().qsa_topk_groups_workspace_size(T, K, score_stride))
+
+
+def qsa_topk_groups(scores, q_pos, K, sel, n_sel, workspace=None, dev_status=None, stream=None):
+    T = scores.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().qsa_topk_groups(
+        _ptr(scores), scores.shape[1], _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel), _ptr(workspace),
+        ws_bytes, _ptr(dev_status), _stream(stream)))
+    return sel, n_sel
+
+
+def qsa_expand_select(sel, n_sel, q_pos, tok, n_tok, capture_pos=None, dev_status=None, stream=None):
+    T, K = sel.shape
+    _check(lib().qsa_expand_select(
+        _ptr(sel), _ptr(n_sel), K, _ptr(q_pos), _ptr(capture_pos), T, _ptr(tok), _ptr(n_tok),
+        tok.shape[1], _ptr(dev_status), _stream(stream)))
+    return tok, n_tok
+
+
+def qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) -> int:
+    return int(lib().qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W))
+
+
+def _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,
+               sm_scale, lse):
+    T, Hq, D = q.shape
+    num_pages, _, Hkv, _ = k_pages.shape
+    return [_ptr(q), _dt(q), _ptr(k_pages), _ptr(v_pages), _dt(k_pages), float(k_scale),
+            float(v_scale), num_pages, _ptr(page_table), page_table.shape[0], page_table.shape[1],
+            _ptr(q_req),
+            _ptr(tok), _ptr(n_tok), tok.shape[1], T, Hq, Hkv, D, float(sm_scale), _ptr(out),
+            _dt(out), _ptr(lse)]
+
+
+def qsa_sparse_attn_decode(q, k_pages, v_pages, page_table, tok, n_tok, out, workspace=None,
+                           k_scale=1.0, v_scale=1.0, q_req=None, sm_scale=0.0, lse=None,
+                           dev_status=None, stream=None):
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    args = _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,
+                      sm_scale, lse)
+    _check(lib().qsa_sparse_attn_decode(*args, _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                        _stream(stream)))
+    return out
+
+
+def qsa_sparse_attn_prefill(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale=1.0,
+                            v_scale=1.0, q_req=None, sm_scale=0.0, lse=None, dev_status=None,
+                            stream=None):
+    args = _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,
+                      sm_scale, lse)
+    _check(lib().qsa_sparse_attn_prefill(*args, _ptr(dev_status), _stream(stream)))
+    return out
+
+
+def qsa_last_error_string() -> str:
+    return lib().qsa_last_error_string().decode()
+
+
+def qsa_abi_version() -> int:
+    return int(lib().qsa_abi_version())

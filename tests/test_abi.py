@@ -1,0 +1,128 @@
+"""The C-ABI library: it builds for sm_100a, loads, exports every entry point
+the header declares, and rejects bad arguments on the host before any launch.
+No GPU needed: every call here fails validation (or has T == 0) before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from indexer_top_sparse_c4_b200 import build, qsa
+    build.build()
+    return qsa.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^QSA_API\s+[\w\s\*]+?\b(qsa_\w+)\s*\(", src, re.M))
+    return sorted(names)
+
+
+def test_header_declares_the_five_calls():
+    names = declared_symbols()
+    for n in ("qsa_index_scores", "qsa_topk_groups", "qsa_expand_select",
+              "qsa_sparse_attn_decode", "qsa_sparse_attn_prefill"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from indexer_top_sparse_c4_b200 import qsa
+    for n in declared_symbols():
+        assert hasattr(L, n), n
+    assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
+    assert L.qsa_abi_version() == 1
+
+
+def test_library_has_no_torch_or_python_dependency():
+    from indexer_top_sparse_c4_b200 import build
+    import subprocess
+    out = subprocess.run(["ldd", build.LIB], capture_output=True, text=True).stdout
+    assert "torch" not in out and "python" not in out and "cudart" not in out
+
+
+def _err(L):
+    return L.qsa_last_error_string().decode()
+
+
+NULL = None
+
+
+def test_index_scores_rejects_unbuilt_shapes(L):
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 3, 128, NULL, 16, NULL, NULL)
+    assert st == 2 and "H_I" in _err(L)
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, -1, 4, 128, NULL, 16, NULL, NULL)
+    assert st == 1
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL)
+    assert st == 1 and "null" in _err(L)
+    st = L.qsa_index_scores(NULL, 2, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL)
+    assert st == 1 and "dtype" in _err(L)
+    # T == 0 is a no-op that launches nothing
+    assert L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 0, 4, 128, NULL, 16, NULL, NULL) == 0
+
+
+def test_index_scores_rejects_misaligned_pointers(L):
+    bad = ctypes.c_void_p(0x1004)
+    ok = ctypes.c_void_p(0x2000)
+    st = L.qsa_index_scores(bad, 0, ok, ok, 0, 1, ok, 1, 1, NULL, ok, 1, 4, 128, ok, 16, NULL, NULL)
+    assert st == 1 and "aligned" in _err(L)
+
+
+def test_topk_validation(L):
+    assert L.qsa_topk_groups(NULL, 16, NULL, 2, 0, NULL, NULL, NULL, 0, NULL, NULL) == 1
+    assert L.qsa_topk_groups(NULL, 0, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 1
+    assert L.qsa_topk_groups(NULL, 10 ** 7, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 2
+    assert L.qsa_topk_groups(NULL, 16, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 0
+    assert L.qsa_topk_groups_workspace_size(8, 512, 65535) == 0
+
+
+def test_expand_validation(L):
+    assert L.qsa_expand_select(NULL, NULL, 8, NULL, NULL, 1, NULL, NULL, 35, NULL, NULL) == 1
+    assert "4*K + 4" in _err(L)
+    assert L.qsa_expand_select(NULL, NULL, 8, NULL, NULL, 1, NULL, NULL, 36, NULL, NULL) == 1
+    assert L.qsa_expand_select(NULL, NULL, 8, NULL, NULL, 0, NULL, NULL, 36, NULL, NULL) == 0
+
+
+def _attn(L, fn, T=1, Hq=16, Hkv=2, D=256, kv_dt=1, q_dt=1, out_dt=1, W=36, ks=1.0, vs=1.0,
+          ptr=NULL, ws=NULL, ws_bytes=0):
+    args = [ptr, q_dt, ptr, ptr, kv_dt, ks, vs, 4, ptr, 1, 1, NULL, ptr, ptr, W, T, Hq, Hkv, D, 0.0, ptr,
+            out_dt, NULL]
+    if fn == "decode":
+        return L.qsa_sparse_attn_decode(*args, ws, ws_bytes, NULL, NULL)
+    return L.qsa_sparse_attn_prefill(*args, NULL, NULL)
+
+
+@pytest.mark.parametrize("fn", ["decode", "prefill"])
+def test_attention_validation(L, fn):
+    assert _attn(L, fn, D=96) == 2 and "head dim" in _err(L)
+    assert _attn(L, fn, Hq=17, Hkv=1) == 2
+    assert _attn(L, fn, Hq=6, Hkv=4) == 1
+    assert _attn(L, fn, kv_dt=2, ks=0.0) == 1 and "FP8" in _err(L)
+    assert _attn(L, fn, q_dt=2) == 1
+    assert _attn(L, fn) == 1 and "null" in _err(L)
+    assert _attn(L, fn, T=0) == 0
+    assert _attn(L, fn, T=70000) == 2
+
+
+def test_decode_workspace_is_checked(L):
+    need = L.qsa_sparse_attn_decode_workspace_size(8, 16, 2, 256, 2052)
+    assert need > 0
+    ok = ctypes.c_void_p(0x10000)
+    st = _attn(L, "decode", T=8, W=2052, ptr=ok, ws=ok, ws_bytes=need - 16)
+    assert st == 3 and str(need) in _err(L)
+
+
+def test_binding_refuses_to_run_without_the_library(monkeypatch, tmp_path):
+    from indexer_top_sparse_c4_b200 import qsa
+    monkeypatch.setattr(qsa, "LIB_PATH", str(tmp_path / "libqsa.so"))
+    monkeypatch.setattr(qsa, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        qsa.lib()

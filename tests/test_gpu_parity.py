@@ -1,0 +1,311 @@
+"""GPU parity: every stage of libqsa.so against the CPU oracle, through the
+C ABI, on the named workloads at full size (sampled rows where the oracle
+would be slow) and on the edge cases of the Ascend operator test list.
+
+Indices (Top-K, expand) are compared bit-exactly on the GPU's own scores;
+scores within the dot-product error bound; attention within the max-abs /
+mean-abs / rel-L2 tolerances against the FP64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from indexer_top_sparse_c4_b200 import workloads as wl
+from indexer_top_sparse_c4_b200.pipeline import QSAStep
+from parity_utils import (ATTN_MAX_ABS, ATTN_MEAN_ABS, ATTN_REL_L2, attn_errors, compact_pages,
+                          host, out_as_f64, score_bound)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from indexer_top_sparse_c4_b200 import build
+    build.build()
+
+
+def _rows(T, n=16):
+    if T <= n:
+        return list(range(T))
+    idx = np.unique(np.linspace(0, T - 1, n).astype(int))
+    return [int(i) for i in idx]
+
+
+def _check_step(oracle, w, step, rows=None, check_scores=True):
+    """Run the four stages on the GPU and compare each with the oracle fed
+    the GPU's previous stage output (scores with their own inputs)."""
+    step.run()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    T = w.T
+    rows = rows if rows is not None else list(range(T))
+    n = {k: host(getattr(w, k)) for k in ("q_idx", "w_idx", "k_idx_pages", "page_table",
+                                         "q_req", "q_pos", "q")}
+    sel_pos = host(step.sel_pos)
+    stride = step.score_stride
+    g_scores = host(step.scores)[rows]
+    # stage 1: scores within the dot-product error bound
+    if check_scores:
+        ref, skipped = oracle.index_scores(n["q_idx"][rows], n["w_idx"][rows], n["k_idx_pages"],
+                                           n["page_table"], sel_pos[rows], n["q_req"][rows], stride)
+        assert skipped == 0
+        bound = score_bound(n["q_idx"], n["w_idx"], n["k_idx_pages"], n["page_table"], n["q_req"],
+                            sel_pos, rows, stride)
+        for i in range(len(rows)):
+            c = min(int(sel_pos[rows[i]]) // 4, stride)
+            err = np.abs(g_scores[i, :c].astype(np.float64) - ref[i, :c])
+            assert np.all(err <= bound[i, :c] + 1e-30), (i, float(err.max()))
+    # stage 2: Top-K bit-exact on the GPU's scores
+    sel_ref, nsel_ref = oracle.topk_groups(np.ascontiguousarray(g_scores), sel_pos[rows], w.K)
+    assert np.array_equal(host(step.n_sel)[rows], nsel_ref)
+    assert np.array_equal(host(step.sel)[rows], sel_ref)
+    # stage 3: expand bit-exact on the GPU's selection
+    cap = None if w.capture_pos is None else host(w.capture_pos)[rows]
+    tok_ref, ntok_ref, bad = oracle.expand_select(host(step.sel)[rows], host(step.n_sel)[rows],
+                                                  n["q_pos"][rows], w.W, cap)
+    assert bad == 0
+    assert np.array_equal(host(step.n_tok)[rows], ntok_ref)
+    assert np.array_equal(host(step.tok)[rows], tok_ref)
+    # stage 4: attention on the GPU's token lists
+    tok = host(step.tok)[rows]
+    ntok = host(step.n_tok)[rows]
+    req = n["q_req"][rows]
+    kc, vc, pt = compact_pages(w.k_pages, w.v_pages, w.page_table, tok, ntok, req)
+    out_ref, lse_ref, sk = oracle.sparse_attn(n["q"][rows], kc, vc, pt, tok, ntok, w.k_scale,
+                                              w.v_scale, q_req=req)
+    assert sk == 0
+    mx, mean, rel = attn_errors(out_as_f64(step.out)[rows], out_ref)
+    assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2, (mx, mean, rel)
+    lse = host(step.lse)[rows].astype(np.float64)
+    assert np.abs(lse - lse_ref).max() < 1e-3
+    return dict(max_abs=mx, mean_abs=mean, rel_l2=rel)
+
+
+def test_tiny_decode(oracle):
+    w = wl.tiny(device="cuda")
+    _check_step(oracle, w, QSAStep(w))
+
+
+def test_b1_decode_16k_bf16(oracle):
+    w = wl.b1_16k(device="cuda")
+    _check_step(oracle, w, QSAStep(w))
+
+
+@pytest.mark.parametrize("K", [512, 1024, 2048])
+def test_b8_decode_262k_fp8(oracle, K):
+    w = wl.b8_262k(K=K, device="cuda")
+    _check_step(oracle, w, QSAStep(w), check_scores=(K == 512))
+
+
+def test_prefill_chunk_sampled_rows(oracle):
+    w = wl.prefill_chunk(device="cuda")
+    step = QSAStep(w, prefill=True)
+    _check_step(oracle, w, step, rows=_rows(w.T, 12))
+
+
+def test_mtp_draft_reuse(oracle):
+    w = wl.mtp(device="cuda")
+    step = QSAStep(w)
+    _check_step(oracle, w, step)
+    tok = host(step.tok)
+    p0 = int(host(w.capture_pos)[0])
+    for t in range(2):   # the group completed since the capture is present
+        assert set(range(p0 - 3, p0 + 1)) <= set(tok[t, : host(step.n_tok)[t]].tolist())
+
+
+SWEEP = [  # every value of every sweep axis appears at least once
+    (4096, 1, (16, 2), 512, "bf16", "ties"),
+    (4096, 8, (3, 1), 2048, "fp8", "normal"),
+    (16384, 2, (12, 1), 1024, "fp8", "peaked"),
+    (16384, 4, (6, 1), 2048, "bf16", "ties"),
+    (65536, 4, (16, 2), 512, "fp8", "normal"),
+    (65536, 1, (3, 1), 1024, "bf16", "peaked"),
+    (131072, 2, (6, 1), 512, "fp8", "ties"),
+    (131072, 8, (12, 1), 2048, "bf16", "normal"),
+    (262144, 1, (16, 2), 2048, "bf16", "ties"),
+    (262144, 2, (12, 1), 1024, "fp8", "peaked"),
+]
+
+
+@pytest.mark.parametrize("case", SWEEP, ids=lambda c: f"c{c[0]}_b{c[1]}_h{c[2][0]}x{c[2][1]}_k{c[3]}_{c[4]}_{c[5]}")
+def test_sweep(oracle, case):
+    ctx, B, heads, K, kv, dist = case
+    w = wl.sweep_case(ctx, B, heads, K, kv, dist, device="cuda", seed=ctx + B)
+    _check_step(oracle, w, QSAStep(w))
+
+
+@pytest.mark.parametrize("dist", ["dyadic", "ties"])
+def test_chain_indices_bit_exact_on_exact_inputs(oracle, dist):
+    """Where every summation order gives the same FP32 score, the whole chain
+    (oracle computing its own scores) selects exactly the GPU's groups."""
+    w = wl.make(f"exact_{dist}", B=4, ctx=65536, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512,
+                kv_dtype="bf16", q_dtype="bf16", dist=dist, seed=21, device="cuda")
+    step = QSAStep(w)
+    step.run()
+    torch.cuda.synchronize()
+    n = w.numpy()
+    r = oracle.qsa_step(n["q"], n["q_idx"], n["w_idx"], n["k_idx_pages"], n["k_pages"], n["v_pages"],
+                        n["page_table"], n["q_pos"], w.K, q_req=n["q_req"])
+    c = int(n["q_pos"][0]) // 4
+    assert np.array_equal(host(step.scores)[:, :c], r["scores"][:, :c])
+    assert np.array_equal(host(step.sel), r["sel"])
+    assert np.array_equal(host(step.tok), r["tok"])
+
+
+def test_chain_on_normal_scores_only_swaps_near_ties(oracle):
+    """Raw N(0,1) inputs: scores differ from the oracle by rounding only, so
+    any index difference must be a swap at the cut within the score bound."""
+    w = wl.make("normal_b8", B=8, ctx=65536, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512,
+                kv_dtype="fp8", q_dtype="bf16", dist="normal", seed=22, device="cuda")
+    step = QSAStep(w)
+    step.run()
+    torch.cuda.synchronize()
+    n = w.numpy()
+    ref, _ = oracle.index_scores(n["q_idx"], n["w_idx"], n["k_idx_pages"], n["page_table"], n["q_pos"],
+                                 n["q_req"], step.score_stride)
+    sel_ref, _ = oracle.topk_groups(ref, n["q_pos"], w.K)
+    bound = score_bound(n["q_idx"], n["w_idx"], n["k_idx_pages"], n["page_table"], n["q_req"],
+                        n["q_pos"], range(w.T), step.score_stride)
+    gsel = host(step.sel)
+    swaps = 0
+    for t in range(w.T):
+        a, b = set(gsel[t].tolist()), set(sel_ref[t].tolist())
+        diff = a ^ b
+        swaps += len(a - b)
+        if diff:
+            kth = np.sort(ref[t][list(b)])[0]
+            for g in diff:
+                assert abs(ref[t, g] - kth) <= 2 * bound[t, g] + 2 * bound[t].max(), (t, g)
+    assert swaps <= w.T * 2
+
+
+# ---- edge cases of the operator test list ------------------------------------------
+
+def _attn_only(oracle, w, tok, n_tok, prefill, sm_scale=0.0, out_dtype=None):
+    step = QSAStep(w, prefill=prefill, out_dtype=out_dtype)
+    step.tok = torch.as_tensor(tok, dtype=torch.int32, device="cuda").contiguous()
+    step.n_tok = torch.as_tensor(n_tok, dtype=torch.int32, device="cuda").contiguous()
+    if not prefill:
+        from indexer_top_sparse_c4_b200 import qsa
+        ws = qsa.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, tok.shape[1])
+        step.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device="cuda")
+    w.W = tok.shape[1]
+    step.attention(sm_scale=sm_scale)
+    torch.cuda.synchronize()
+    n = w.numpy()
+    ref, lse, sk = oracle.sparse_attn(n["q"], host(w.k_pages), host(w.v_pages), n["page_table"], tok,
+                                      n_tok, w.k_scale, w.v_scale, q_req=n["q_req"], sm_scale=sm_scale)
+    return step, ref, lse, sk
+
+
+@pytest.mark.parametrize("width", [1, 63, 64, 65, 2051])
+@pytest.mark.parametrize("prefill", [False, True])
+def test_unordered_slots_of_any_width(oracle, width, prefill):
+    w = wl.make("slots", B=2, ctx=8192, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="bf16",
+                q_dtype="bf16", seed=width, device="cuda", q_pos=[8191, 5000], q_req=[0, 1])
+    rng = np.random.default_rng(width)
+    tok = np.stack([rng.permutation(8192)[:width], rng.permutation(5001)[:width]]).astype(np.int32)
+    step, ref, lse, sk = _attn_only(oracle, w, tok, np.array([width, width]), prefill)
+    mx, mean, rel = attn_errors(out_as_f64(step.out), ref)
+    assert sk == 0 and mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2
+
+
+@pytest.mark.parametrize("sm_scale", [0.0, 0.03125, 0.2])
+def test_default_and_explicit_scale(oracle, sm_scale):
+    w = wl.make("scale", B=1, ctx=4096, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="fp8",
+                q_dtype="bf16", seed=3, device="cuda")
+    tok = np.arange(0, 4096, 3, dtype=np.int32)[None]
+    step, ref, lse, _ = _attn_only(oracle, w, tok, np.array([tok.shape[1]]), False, sm_scale)
+    mx, mean, rel = attn_errors(out_as_f64(step.out), ref)
+    assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2
+    assert np.abs(host(step.lse) - lse).max() < 1e-3
+
+
+@pytest.mark.parametrize("prefill", [False, True])
+def test_masked_and_zero_rows_are_exact_zero(oracle, prefill):
+    w = wl.make("empty", B=3, ctx=1024, Hq=6, Hkv=1, D=256, H_I=4, D_I=128, K=64, kv_dtype="bf16",
+                q_dtype="bf16", seed=4, device="cuda", q_pos=[1023, 1023, 1023], q_req=[0, 1, 2])
+    tok = np.full((3, 64), -1, np.int32)
+    tok[2, :5] = [1, 2, 3, 700, 1023]
+    n_tok = np.array([64, 0, 5])          # all -1 / width 0 / normal
+    step, ref, lse, _ = _attn_only(oracle, w, tok, n_tok, prefill)
+    out = out_as_f64(step.out)
+    assert np.all(out[:2] == 0) and np.all(host(step.lse)[:2] == -np.inf)
+    assert attn_errors(out[2:], ref[2:])[0] <= ATTN_MAX_ABS
+
+
+@pytest.mark.parametrize("rem", [0, 1, 2, 3])
+def test_causal_tail_remainders(oracle, rem):
+    """p % 4 = 0..3: the current block holds 1..4 tokens and always the query."""
+    p = 4 * 1000 + rem
+    w = wl.make("tail", B=1, ctx=p + 1, Hq=12, Hkv=1, D=256, H_I=4, D_I=128, K=128, kv_dtype="bf16",
+                q_dtype="bf16", seed=rem, device="cuda")
+    step = QSAStep(w)
+    _check_step(oracle, w, step)
+    row = host(step.tok)[0, : host(step.n_tok)[0]]
+    assert row[-1] == p and list(row[-(rem + 1):]) == list(range(4 * 1000, p + 1))
+
+
+def test_selection_width_zero_before_first_group(oracle):
+    """p < 4: no complete group, n_sel = 0, only the current block is attended."""
+    w = wl.make("w0", B=3, ctx=64, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=8, kv_dtype="bf16",
+                q_dtype="bf16", seed=5, device="cuda", q_pos=[0, 2, 3], q_req=[0, 1, 2])
+    step = QSAStep(w)
+    _check_step(oracle, w, step)
+    assert host(step.n_sel).tolist() == [0, 0, 0]
+    assert host(step.n_tok).tolist() == [1, 3, 4]
+
+
+def test_two_requests_sharing_prefix_pages(oracle):
+    w = wl.make("shared", B=2, ctx=8192, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=256, kv_dtype="fp8",
+                q_dtype="bf16", seed=6, device="cuda")
+    w.page_table[1, :64] = w.page_table[0, :64]     # first 4,096 tokens shared
+    w.q_idx[1] = w.q_idx[0]
+    w.w_idx[1] = w.w_idx[0]
+    step = QSAStep(w)
+    _check_step(oracle, w, step)
+
+
+def test_cache_content_reuse_is_deterministic():
+    w = wl.b1_16k(device="cuda", seed=7)
+    step = QSAStep(w)
+    step.run()
+    a = [t.clone() for t in (step.scores, step.sel, step.tok, step.out, step.lse)]
+    step.run()
+    torch.cuda.synchronize()
+    for x, y in zip(a, (step.scores, step.sel, step.tok, step.out, step.lse)):
+        assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("heads", [(16, 2), (24, 2), (12, 1), (6, 1), (3, 1)])
+@pytest.mark.parametrize("T", [1, 257])
+def test_local_head_shapes_prefill_rows(oracle, heads, T):
+    Hq, Hkv = heads
+    ctx = 16384
+    pos = np.sort(np.random.default_rng(T).integers(8000, ctx, T)).astype(np.int32)
+    w = wl.make("heads", B=1, ctx=ctx, Hq=Hq, Hkv=Hkv, D=256, H_I=4, D_I=128, K=512, kv_dtype="bf16",
+                q_dtype="bf16", seed=Hq * T, device="cuda", q_pos=pos, q_req=np.zeros(T, np.int32))
+    step = QSAStep(w, prefill=True)
+    _check_step(oracle, w, step, rows=_rows(T, 6))
+
+
+def test_bad_page_id_is_flagged_not_trapped():
+    from indexer_top_sparse_c4_b200 import qsa
+    w = wl.make("bad", B=1, ctx=4096, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=64, kv_dtype="bf16",
+                q_dtype="bf16", seed=8, device="cuda")
+    w.page_table[0, 5] = 10 ** 6
+    step = QSAStep(w)
+    step.run()
+    torch.cuda.synchronize()
+    st = int(step.status.item())
+    assert st & qsa.QSA_DEV_BAD_PAGE
+    assert torch.isfinite(step.out.float()).all()
+
+
+def test_non_contiguous_input_is_refused():
+    w = wl.tiny(device="cuda")
+    step = QSAStep(w)
+    w.q_idx = w.q_idx.transpose(1, 2)
+    with pytest.raises(ValueError, match="contiguous"):
+        step.index_scores()
