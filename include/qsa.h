@@ -165,6 +165,31 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, co
                                      float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
                                      uint32_t* dev_status, qsa_stream_t stream);
 
+/* qsa_sparse_attn_decode without a workspace argument, for callers that cannot
+ * allocate device memory: code recorded into a CUDA graph that must not
+ * allocate, code running under a memory pool that is already fully carved up,
+ * or a plugin layer that is handed only its input and output buffers.  (The
+ * pages have no counterpart: this is a deployment convenience of this
+ * library, not part of the method.)
+ * Same arguments, results and checks as qsa_sparse_attn_decode.  The split-K
+ * scratch lives in a fixed array of QSA_DECODE_NOALLOC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads libqsa.so keeps until the process
+ * exits; a shape whose scratch (qsa_sparse_attn_decode_workspace_size) is
+ * larger is refused with QSA_ERR_WORKSPACE.  The call allocates nothing.
+ * The first call on a device looks up that device's copy of the array
+ * (cudaGetSymbolAddress, with the device current): make that first call
+ * before any stream capture on the device.  Every call shares the one array
+ * and every kernel overwrites all the scratch it later reads, so nothing
+ * needs clearing; but calls whose kernels overlap on the GPU (two streams, or
+ * two host threads) race on it -- serialise them. */
+#define QSA_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
+    const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages, qsa_dtype_t kv_dt,
+    float k_scale, float v_scale, int num_pages, const int32_t* page_table, int pt_rows,
+    int pt_stride, const int32_t* q_req, const int32_t* tok, const int32_t* n_tok, int W, int T,
+    int Hq, int Hkv, int D, float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+    uint32_t* dev_status, qsa_stream_t stream);
+
 /* Human-readable message for the last non-OK status returned on this thread. */
 QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */

@@ -65,6 +65,8 @@ qsa_status_t check_attn(const void* q, qsa_dtype_t q_dt, const void* k_pages, co
 
 }  // namespace
 
+void qsa::set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+
 extern "C" {
 
 const char* qsa_last_error_string(void) { return g_err; }

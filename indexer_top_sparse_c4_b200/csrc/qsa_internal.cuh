@@ -143,4 +143,7 @@ int attn_decode_splits(int T, int Hkv, int W);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
 cudaError_t launch_sparse_attn(const AttnArgs& a, int splits, void* ws, cudaStream_t s);
 
+// Sets the message qsa_last_error_string() returns on this thread.
+void set_last_error(const char* msg);
+
 }  // namespace qsa

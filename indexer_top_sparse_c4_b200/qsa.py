@@ -179,3 +179,22 @@ def qsa_last_error_string() -> str:
 
 def qsa_abi_version() -> int:
     return int(lib().qsa_abi_version())
+
+
+def qsa_sparse_attn_decode_noalloc(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale=1.0,
+                                   v_scale=1.0, q_req=None, sm_scale=0.0, lse=None,
+                                   dev_status=None, stream=None):
+    """qsa_sparse_attn_decode without a workspace: for callers that cannot
+    allocate device memory.  The library's own fixed scratch buffer is used
+    (QSA_DECODE_NOALLOC_SCRATCH_BYTES per device); larger shapes raise
+    QSAError(QSA_ERR_WORKSPACE).  Calls that overlap on the GPU share that
+    buffer and must not run concurrently."""
+    fn = lib().qsa_sparse_attn_decode_noalloc
+    if fn.argtypes is None:
+        P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        fn.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I, F, P, I, P, P, P]
+        fn.restype = I
+    args = _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,
+                      sm_scale, lse)
+    _check(fn(*args, _ptr(dev_status), _stream(stream)))
+    return out

@@ -1,0 +1,70 @@
+"""qsa_sparse_attn_decode_noalloc: the decode attention for callers that cannot
+allocate device memory (a graph capture that must not allocate, a fully
+carved-up memory pool, a plugin handed only its inputs and outputs).  It must
+give the same results as qsa_sparse_attn_decode with a caller workspace, call
+after call, although every call reuses the library's one scratch buffer.
+
+Kept in a file of its own that pytest collects last."""
+import numpy as np
+import pytest
+import torch
+
+from parity_utils import ATTN_MAX_ABS, ATTN_MEAN_ABS, ATTN_REL_L2, attn_errors
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from indexer_top_sparse_c4_b200 import build, qsa
+    build.build()
+    return qsa
+
+
+def _selection(w):
+    from indexer_top_sparse_c4_b200.pipeline import QSAStep
+    step = QSAStep(w)
+    step.run()                       # decode through the workspace entry point
+    torch.cuda.synchronize()
+    return step
+
+
+@pytest.mark.parametrize("which", ["b8_262k_fp8", "b1_16k_bf16"])
+def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
+    from indexer_top_sparse_c4_b200 import workloads as wl
+    make = (lambda s: wl.b8_262k(K=512, device="cuda", seed=s)) if which == "b8_262k_fp8" else \
+        (lambda s: wl.b1_16k(device="cuda", seed=s))
+    for seed in (11, 12):            # two calls in a row, different inputs each time
+        w = make(seed)
+        step = _selection(w)
+        need = lib.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, w.W)
+        assert 0 < need <= 8 * 1024 * 1024
+        out = torch.full_like(step.out, float("nan"))
+        lse = torch.full_like(step.lse, float("nan"))
+        status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        lib.qsa_sparse_attn_decode_noalloc(w.q, w.k_pages, w.v_pages, w.page_table, step.tok,
+                                           step.n_tok, out, k_scale=w.k_scale, v_scale=w.v_scale,
+                                           q_req=w.q_req, lse=lse, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        ref = step.out.double().cpu().numpy()
+        got = out.double().cpu().numpy()
+        mx, mean, rel = attn_errors(got, ref)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2, (mx, mean, rel)
+        assert torch.allclose(lse, step.lse, atol=1e-3, rtol=0)
+
+
+def test_noalloc_refuses_shapes_beyond_its_buffer(lib):
+    # 64 queries x 16 heads x 10 splits of 256-float partials do not fit in 8 MiB
+    T, Hq, Hkv, D, W = 64, 16, 1, 256, 2052
+    assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) > 8 * 1024 * 1024
+    q = torch.zeros((T, Hq, D), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")
+    pt = torch.zeros((T, 1), dtype=torch.int32, device="cuda")
+    tok = torch.full((T, W), -1, dtype=torch.int32, device="cuda")
+    n_tok = torch.zeros((T,), dtype=torch.int32, device="cuda")
+    out = torch.empty((T, Hq, D), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.QSAError, match="built-in buffer"):
+        lib.qsa_sparse_attn_decode_noalloc(q, kv, kv, pt, tok, n_tok, out, k_scale=1.0, v_scale=1.0)
