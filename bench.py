@@ -33,7 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QSA sparse-decode tokens/s @B8×262K FP8 KV; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS_PER_STEP = 5  # index, topk, expand, attention, split-K combine
+KERNELS_PER_STEP = 4  # index, topk, expand, attention (partials merged inside the attention clusters)
 
 
 def peak_hbm():
@@ -138,52 +138,90 @@ class ClockSampler:
 
 # ---- the GPU arm -----------------------------------------------------------------------
 
-def make_sets(K, device, seed, n_sets=2):
+def make_sets(K, device, seed, n_sets=2, context=262144):
     from indexer_top_sparse_c4_b200 import workloads as wl
     from indexer_top_sparse_c4_b200.pipeline import QSAStep
     sets = []
     for i in range(n_sets):
-        w = wl.b8_262k(K=K, device=device, seed=seed + i)
+        w = wl.b8_262k(K=K, device=device, seed=seed + i, ctx=context)
         sets.append(QSAStep(w))
     return sets
 
 
-def time_steps(sets, steps, warmup, stream):
-    """Per-step and per-stage CUDA-event times (ms) over `steps` timed steps."""
-    for i in range(warmup):
-        sets[i % len(sets)].run(stream)
-    torch.cuda.synchronize()
-    barrier()
-    torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        start.record(stream)
+STAGES = ("index_scores", "topk", "expand", "attention")
+STAGE_NAMES = ("index_scores", "topk_groups", "expand_select", "sparse_attn_decode")
+
+
+def capture(sets, steps, stages=STAGES):
+    """One CUDA graph of `steps` consecutive QSA steps (alternating input
+    sets), each step the given stages in order."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
         for i in range(steps):
             st = sets[i % len(sets)]
-            e = ev[i]
-            e[0].record(stream)
-            st.index_scores(stream)
-            e[1].record(stream)
-            st.topk(stream)
-            e[2].record(stream)
-            st.expand(stream)
-            e[3].record(stream)
-            st.attention(stream)
-            e[4].record(stream)
-        end.record(stream)
+            for name in stages:
+                getattr(st, name)()
+    return g
+
+
+def replay_ms(g):
+    """Device time of one replay of `g` (CUDA events on the current stream)."""
     torch.cuda.synchronize()
     barrier()
-    total = start.elapsed_time(end)
-    stages = np.array([[e[j].elapsed_time(e[j + 1]) for j in range(4)] for e in ev])
-    return total, stages.mean(axis=0)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    g.replay()
+    end.record()
+    torch.cuda.synchronize()
+    barrier()
+    return start.elapsed_time(end)
+
+
+def time_steps(sets, steps, warmup, stream):
+    """Device time (ms) of exactly `steps` steps replayed from one CUDA graph,
+    after `warmup` eager steps and one untimed replay."""
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            sets[i % len(sets)].run()
+        torch.cuda.synchronize()
+        g = capture(sets, steps)
+        g.replay()
+        total = replay_ms(g)
+    del g
+    return total
+
+
+def time_stages(sets, reps, stream):
+    """Per-stage device times (us).  `alone`: a graph of `reps` launches of that
+    stage only (for the indexer scan every launch streams its 256 MiB of keys
+    from HBM, so this is its true launch duration).  `in_step`: what the stage
+    adds to a step, i.e. the step graph minus the same graph without it."""
+    alone, in_step = {}, {}
+    with torch.cuda.stream(stream):
+        full = capture(sets, reps)
+        full.replay()
+        t_full = replay_ms(full)
+        del full
+        for name in STAGES:
+            g = capture(sets, reps, (name,))
+            g.replay()
+            alone[name] = replay_ms(g) / reps * 1e3
+            del g
+            g = capture(sets, reps, tuple(x for x in STAGES if x != name))
+            g.replay()
+            in_step[name] = (t_full - replay_ms(g)) / reps * 1e3
+            del g
+    return alone, in_step
 
 
 def time_e2e(sets, steps, warmup, stream):
-    """Through the public API with host buffers: per step, copy the step's
-    query-side inputs from pinned host memory, run the four calls, read the
-    output back.  The KV cache and indexer keys are resident device state."""
+    """Through the public API with host buffers: every step copies its
+    query-side inputs from pinned host memory to the device, runs the four
+    calls and copies the output back to pinned host memory; the steps are
+    captured once as CUDA graphs (one per input set) and replayed.  The KV
+    cache and the indexer keys are resident device state."""
     hosts = []
     for st in sets:
         w = st.w
@@ -198,20 +236,29 @@ def time_e2e(sets, steps, warmup, stream):
         hin, dev_in, hout = hosts[i % len(sets)]
         for h, d in zip(hin, dev_in):
             d.copy_(h, non_blocking=True)
-        st.run(stream)
+        st.run()
         hout.copy_(st.out, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(warmup):
             one(i)
         torch.cuda.synchronize()
+        graphs = []
+        for i in range(len(sets)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                one(i)
+            graphs.append(g)
+        for g in graphs:
+            g.replay()
+        torch.cuda.synchronize()
         barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+        a.record()
         for i in range(steps):
-            one(i)
-        b.record(stream)
+            graphs[i % len(graphs)].replay()
+        b.record()
     torch.cuda.synchronize()
     barrier()
     return a.elapsed_time(b), h2d, d2h
@@ -231,13 +278,14 @@ def gpu_arm(args):
         build.build()
     barrier()
     stream = torch.cuda.Stream(device)
-    sets = make_sets(args.budget, device, rank_seed(args.seed, rank))
+    sets = make_sets(args.budget, device, rank_seed(args.seed, rank), context=args.context)
     w0 = sets[0].w
     with ClockSampler(local) as clk:
-        total_ms, stages = time_steps(sets, args.steps, args.warmup, stream)
+        total_ms = time_steps(sets, args.steps, args.warmup, stream)
+        alone, in_step = time_stages(sets, 40, stream)
+        e2e_ms, h2d, d2h = time_e2e(sets, args.steps, args.warmup, stream)
     total_ms = reduce_max(total_ms, device)
     ms = total_ms / args.steps
-    e2e_ms, h2d, d2h = time_e2e(sets, args.steps, args.warmup, stream)
     e2e_ms = reduce_max(e2e_ms, device)
     n_tok_total = int(sets[0].n_tok.sum().item())
     idx_bytes, kv_bytes = algorithmic_bytes(w0, n_tok_total)
@@ -249,8 +297,8 @@ def gpu_arm(args):
                 continue
             del sets
             torch.cuda.empty_cache()
-            sets = make_sets(K, device, rank_seed(args.seed, rank))
-            t, _ = time_steps(sets, max(3, args.steps // 2), args.warmup, stream)
+            sets = make_sets(K, device, rank_seed(args.seed, rank), context=args.context)
+            t = time_steps(sets, max(3, args.steps // 2), args.warmup, stream)
             t = reduce_max(t, device) / max(3, args.steps // 2)
             nt = int(sets[0].n_tok.sum().item())
             ib, kb = algorithmic_bytes(sets[0].w, nt)
@@ -260,7 +308,7 @@ def gpu_arm(args):
     if rank != 0:
         return None
     peak, peak_kind = peak_hbm()
-    idx_ms = float(stages[0])
+    idx_ms = alone["index_scores"] / 1e3
     idx_gbs = idx_bytes / (idx_ms / 1e3) / 1e9
     step_gbs = (idx_bytes + kv_bytes) / (ms / 1e3) / 1e9
     value = ws * w0.B / (ms / 1e3)
@@ -269,7 +317,7 @@ def gpu_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
-        "config": {"workload": w0.name, "B": w0.B, "context": 262144, "Hq": w0.Hq, "Hkv": w0.Hkv,
+        "config": {"workload": w0.name, "B": w0.B, "context": args.context, "Hq": w0.Hq, "Hkv": w0.Hkv,
                    "D": w0.D, "H_I": w0.H_I, "D_I": w0.D_I, "budget_groups": w0.K,
                    "kv_storage": "fp8_e4m3 per-tensor scale", "indexer_keys": "fp32, peaked (5% +3 sigma)",
                    "page_table": "random permutation, page size 64",
@@ -282,12 +330,12 @@ def gpu_arm(args):
         "step_hbm": {"achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(step_gbs / peak, 4), "bytes_per_step": idx_bytes + kv_bytes,
                      "indexer_key_bytes": idx_bytes, "selected_kv_bytes": kv_bytes},
-        "stages_us": {k: round(float(v) * 1e3, 2) for k, v in
-                      zip(("index_scores", "topk_groups", "expand_select", "sparse_attn_decode"), stages)},
+        "stages_us": {"alone": {n: round(alone[k], 2) for n, k in zip(STAGE_NAMES, STAGES)},
+                      "in_step": {n: round(in_step[k], 2) for n, k in zip(STAGE_NAMES, STAGES)}},
         "e2e": {"value": round(ws * w0.B / (e2e_ms / args.steps / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms / args.steps, 5)},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": (KERNELS_PER_STEP + (1 if sets[0].ws_bytes else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     if budgets:
@@ -365,6 +413,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--budget", type=int, default=512, help="budget in groups (512, 1024, 2048)")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--context", type=int, default=262144,
+                    help="tokens per request; smaller values give the small cases used for profiling")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--all-budgets", action="store_true", default=True)
     ap.add_argument("--headline-only", dest="all_budgets", action="store_false")

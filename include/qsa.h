@@ -182,7 +182,7 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, co
  * and every kernel overwrites all the scratch it later reads, so nothing
  * needs clearing; but calls whose kernels overlap on the GPU (two streams, or
  * two host threads) race on it -- serialise them. */
-#define QSA_DECODE_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
+#define QSA_DECODE_NOALLOC_SCRATCH_BYTES (512u * 1024u)
 QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
     const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages, qsa_dtype_t kv_dt,
     float k_scale, float v_scale, int num_pages, const int32_t* page_table, int pt_rows,

@@ -15,9 +15,10 @@ namespace {
 constexpr int kThreads = 256;
 
 __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandArgs a) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int t = blockIdx.y;
   const int p = a.q_pos[t];
-  const int c = p >= 0 ? p / kGroupTokens : 0;
   int p0 = a.capture_pos ? a.capture_pos[t] : p;
   if (p0 > p) p0 = p;
   const int c0 = p0 >= 0 ? p0 / kGroupTokens : 0;
@@ -51,8 +52,7 @@ cudaError_t launch_expand_select(const ExpandArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
   int bx = (a.W + kThreads - 1) / kThreads;
   if (bx > 64) bx = 64;
-  expand_kernel<<<dim3(bx, a.T), kThreads, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(expand_kernel, dim3(bx, a.T), dim3(kThreads), 0, s, 1, a);
 }
 
 }  // namespace qsa

@@ -54,6 +54,8 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
   const int t = blockIdx.y;
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  pdl_wait();
+  pdl_launch_dependents();  // the next kernel's CTAs may take SMs this grid's last wave leaves free
   const int p = a.q_pos[t];
   int c = p >= 0 ? p / kGroupTokens : 0;
   if (c > a.score_stride) {
@@ -124,8 +126,8 @@ cudaError_t launch_typed(const IndexArgs& a, cudaStream_t s) {
   const int blocks = (warps_per_row + kWarps - 1) / kWarps;
   warps_per_row = blocks * kWarps;
   dim3 grid(blocks, a.T);
-  index_scores_kernel<H_I, D_I, QT, KT><<<grid, kThreads, 0, s>>>(a, warps_per_row);
-  return cudaGetLastError();
+  return launch_k(index_scores_kernel<H_I, D_I, QT, KT>, grid, dim3(kThreads), 0, s, 1, a,
+                  warps_per_row);
 }
 
 template <int H_I, int D_I>

@@ -8,6 +8,8 @@
 #include <cuda_fp8.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/qsa.h"
 
 namespace qsa {
@@ -108,6 +110,45 @@ __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// ---- programmatic dependent launch (PDL) ----------------------------------------
+// Every kernel of the library is launched with programmatic stream
+// serialisation, so its CTAs may be scheduled while the previous kernel on the
+// stream is still finishing.  pdl_wait() blocks until that kernel has
+// completed and its memory is visible; a kernel calls it before its first
+// access to global memory (it returns at once when there is no such kernel).
+// pdl_launch_dependents() lets the next kernel's CTAs be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch `kern` on `s` with PDL enabled and, when cluster > 1, a
+// (cluster, 1, 1) thread-block cluster.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t s, int cluster, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---- launchers (one per stage; defined in the stage's .cu file) -----------------
 
 struct IndexArgs {
@@ -137,11 +178,19 @@ struct AttnArgs {
   const int32_t* q_req; const int32_t* tok; const int32_t* n_tok; int W, T, Hq, Hkv, D;
   float sm_scale; void* out; qsa_dtype_t out_dt; float* lse; uint32_t* status;
 };
-// splits > 1: partial (o, m, l) per split go to ws_o / ws_ml and a combine
-// kernel finishes; splits == 1 writes out / lse directly.
-int attn_decode_splits(int T, int Hkv, int W);
+// How a decode call is spread over the GPU: clusters of `cl` CTAs per
+// (query, KV head) merged on chip, and `s` cluster groups whose partial
+// (o, max, sum) go through the workspace to the combine kernel when s > 1.
+struct DecodePlan { int cl, s; };
+DecodePlan attn_decode_plan(int T, int Hkv, int W);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
-cudaError_t launch_sparse_attn(const AttnArgs& a, int splits, void* ws, cudaStream_t s);
+cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s);
+
+// Tensor-core decode kernel (BF16 / FP8 caches, D in {128, 256}, <= 8 query
+// heads per KV head); same partial / output contract as the general kernel.
+bool attn_mma_supported(const AttnArgs& a);
+cudaError_t launch_sparse_attn_mma(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
+                                   int s, void* ws, cudaStream_t stream);
 
 // Sets the message qsa_last_error_string() returns on this thread.
 void set_last_error(const char* msg);

@@ -161,6 +161,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, AttnSca
 template <typename OT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs a, AttnScales sc, int splits,
                                                            const float* ws_o, const float* ws_ml) {
+  pdl_wait();
   const size_t th = blockIdx.x;
   const float* ml = ws_ml + th * splits * 2;
   float M = -INFINITY;
@@ -191,10 +192,19 @@ cudaError_t launch_typed(const AttnArgs& a, const AttnScales& sc, int splits, vo
   float* ws_o = reinterpret_cast<float*>(ws);
   float* ws_ml = ws_o ? ws_o + (size_t)a.T * a.Hq * splits * D : nullptr;
   kern<<<dim3(splits, a.Hkv, a.T), kThreads, smem, s>>>(a, sc, splits, chunk, ws_o, ws_ml);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || splits == 1) return e;
-  attn_combine_kernel<OT><<<a.T * a.Hq, D < 256 ? D : 256, 0, s>>>(a, sc, splits, ws_o, ws_ml);
   return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const AttnArgs& a, const AttnScales& sc, int splits, void* ws,
+                           cudaStream_t s) {
+  const float* ws_o = reinterpret_cast<const float*>(ws);
+  const float* ws_ml = ws_o + (size_t)a.T * a.Hq * splits * a.D;
+  const int threads = a.D < 256 ? a.D : 256;
+  if (a.out_dt == QSA_F32)
+    return launch_k(attn_combine_kernel<float>, dim3(a.T * a.Hq), dim3(threads), 0, s, 1, a, sc,
+                    splits, ws_o, ws_ml);
+  return launch_k(attn_combine_kernel<__nv_bfloat16>, dim3(a.T * a.Hq), dim3(threads), 0, s, 1, a,
+                  sc, splits, ws_o, ws_ml);
 }
 
 template <int D, typename QT, typename KVT>
@@ -220,13 +230,20 @@ cudaError_t launch_q(const AttnArgs& a, const AttnScales& sc, int splits, void* 
 
 }  // namespace
 
-int attn_decode_splits(int T, int Hkv, int W) {
-  // enough CTAs to cover the 148 SMs several times, at least 32 tokens each
+DecodePlan attn_decode_plan(int T, int Hkv, int W) {
+  // CTAs per (query, KV head): a power of two, at most 128 CTAs in all and at
+  // least one 128-token round each.  With one CTA per SM (the tensor-core
+  // kernel's shared memory) at most 33 clusters of 4 fit on the GPU at once,
+  // so clusters stay <= 4 and every cluster is resident in a single wave;
+  // cluster groups beyond that merge through the workspace.
   const int rows = T * Hkv > 0 ? T * Hkv : 1;
-  int splits = (4 * 148 + rows - 1) / rows;
-  const int max_splits = (W + 31) / 32;
-  if (splits > max_splits) splits = max_splits;
-  return splits < 1 ? 1 : splits;
+  const int tiles = (W + 15) / 16;
+  int per = 1;
+  while (per < 64 && per * 2 * rows <= 128 && per * 2 * 8 <= tiles) per <<= 1;
+  DecodePlan p;
+  p.cl = per < 4 ? per : 4;
+  p.s = per / p.cl;
+  return p;
 }
 
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
@@ -234,19 +251,27 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
   return (size_t)T * Hq * splits * (D + 2) * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const AttnArgs& a, int splits, void* ws, cudaStream_t s) {
+cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s) {
+  const int splits = plan.s;
   if (a.T == 0) return cudaSuccess;
   const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
   const bool fp8 = a.kv_dt == QSA_FP8_E4M3;
   AttnScales sc;
   sc.qk = (float)(scale * 1.4426950408889634 * (fp8 ? (double)a.k_scale : 1.0));
   sc.vmul = fp8 ? a.v_scale : 1.f;
-  switch (a.D) {
-    case 64: return launch_q<64>(a, sc, splits, ws, s);
-    case 128: return launch_q<128>(a, sc, splits, ws, s);
-    case 256: return launch_q<256>(a, sc, splits, ws, s);
-    default: return cudaErrorInvalidValue;
+  cudaError_t e;
+  if (attn_mma_supported(a)) {
+    e = launch_sparse_attn_mma(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
+  } else {
+    switch (a.D) {
+      case 64: e = launch_q<64>(a, sc, splits, ws, s); break;
+      case 128: e = launch_q<128>(a, sc, splits, ws, s); break;
+      case 256: e = launch_q<256>(a, sc, splits, ws, s); break;
+      default: return cudaErrorInvalidValue;
+    }
   }
+  if (e != cudaSuccess || splits == 1) return e;
+  return launch_combine(a, sc, splits, ws, s);
 }
 
 }  // namespace qsa

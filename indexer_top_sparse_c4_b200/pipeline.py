@@ -37,6 +37,7 @@ class QSAStep:
         self.lse = torch.empty((T, w.Hq), dtype=torch.float32, device=dev)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
         ws = 0 if self.prefill else qsa.qsa_sparse_attn_decode_workspace_size(T, w.Hq, w.Hkv, w.D, w.W)
+        self.ws_bytes = ws   # > 0: split-K partials and one combine kernel per call
         self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
         tk = qsa.qsa_topk_groups_workspace_size(T, w.K, self.score_stride)
         self.topk_ws = torch.empty((max(tk, 16),), dtype=torch.uint8, device=dev) if tk else None

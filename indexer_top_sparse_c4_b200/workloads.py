@@ -240,7 +240,8 @@ def b8_262k(K=512, device="cpu", seed=0, **kw) -> Workload:
     args = dict(B=8, ctx=262144, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=K, kv_dtype="fp8",
                 q_dtype="bf16", dist="peaked", pages="perm", seed=seed, device=device)
     args.update(kw)
-    return make(f"b8_decode_262k_fp8_k{args['K']}", **args)
+    name = "262k" if args["ctx"] == 262144 else f"{args['ctx']}"
+    return make(f"b8_decode_{name}_fp8_k{args['K']}", **args)
 
 
 def prefill_chunk(device="cpu", seed=0, new=8192, prefix=57344, **kw) -> Workload:

@@ -31,16 +31,16 @@ def _selection(w):
     return step
 
 
-@pytest.mark.parametrize("which", ["b8_262k_fp8", "b1_16k_bf16"])
+@pytest.mark.parametrize("which", ["b1_16k_bf16", "b2_16k_fp8"])
 def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
     from indexer_top_sparse_c4_b200 import workloads as wl
-    make = (lambda s: wl.b8_262k(K=512, device="cuda", seed=s)) if which == "b8_262k_fp8" else \
-        (lambda s: wl.b1_16k(device="cuda", seed=s))
+    make = (lambda s: wl.b1_16k(device="cuda", seed=s)) if which == "b1_16k_bf16" else \
+        (lambda s: wl.b1_16k(device="cuda", seed=s, B=2, kv_dtype="fp8"))
     for seed in (11, 12):            # two calls in a row, different inputs each time
         w = make(seed)
         step = _selection(w)
         need = lib.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, w.W)
-        assert 0 < need <= 8 * 1024 * 1024
+        assert 0 < need <= 512 * 1024       # small batches split across CTAs: scratch in use
         out = torch.full_like(step.out, float("nan"))
         lse = torch.full_like(step.lse, float("nan"))
         status = torch.zeros((1,), dtype=torch.int32, device="cuda")
@@ -57,9 +57,9 @@ def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
 
 
 def test_noalloc_refuses_shapes_beyond_its_buffer(lib):
-    # 64 queries x 16 heads x 10 splits of 256-float partials do not fit in 8 MiB
-    T, Hq, Hkv, D, W = 64, 16, 1, 256, 2052
-    assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) > 8 * 1024 * 1024
+    # 16 queries x 16 heads x 2 split groups of 256-float partials exceed 512 KiB
+    T, Hq, Hkv, D, W = 16, 16, 1, 256, 2052
+    assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) > 512 * 1024
     q = torch.zeros((T, Hq, D), dtype=torch.bfloat16, device="cuda")
     kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")
     pt = torch.zeros((T, 1), dtype=torch.int32, device="cuda")
