@@ -142,10 +142,14 @@ QSA_API qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel,
  * sm_scale <= 0.  lse may be NULL.
  * Supported: D in {64, 128, 256}, Hq/Hkv <= 16, q_dt F32 or BF16, kv_dt F32,
  * BF16 or FP8_E4M3, out_dt F32 or BF16.
- * _decode splits every row's tokens across CTAs (split-K) and needs
- * qsa_sparse_attn_decode_workspace_size() bytes of workspace; _prefill
- * gives each (query, KV head) its own CTA and needs no workspace. */
-QSA_API size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W);
+ * _decode splits every row's tokens across CTAs (split-K): the CTAs of a
+ * thread-block cluster merge their partials on chip; when a call needs more
+ * than one cluster per (query, KV head) the clusters' partials go through
+ * qsa_sparse_attn_decode_workspace_size(..., kv_dt) bytes of workspace (0 when
+ * none is needed).  _prefill gives each (query, KV head) its own CTA and needs
+ * no workspace. */
+QSA_API size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W,
+                                                     qsa_dtype_t kv_dt);
 QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
                                     const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
                                     float v_scale, int num_pages, const int32_t* page_table,
@@ -182,7 +186,7 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, co
  * and every kernel overwrites all the scratch it later reads, so nothing
  * needs clearing; but calls whose kernels overlap on the GPU (two streams, or
  * two host threads) race on it -- serialise them. */
-#define QSA_DECODE_NOALLOC_SCRATCH_BYTES (512u * 1024u)
+#define QSA_DECODE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
     const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages, qsa_dtype_t kv_dt,
     float k_scale, float v_scale, int num_pages, const int32_t* page_table, int pt_rows,
@@ -194,7 +198,8 @@ QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
 QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */
 QSA_API const char* qsa_status_name(qsa_status_t s);
-/* ABI version: bumped on any signature change. */
+/* ABI version: bumped on any signature change (2: the decode workspace query
+ * takes the KV dtype). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -61,7 +61,7 @@ qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, qsa_dtype_t q_dt, con
                                             int D, float sm_scale, void* out, qsa_dtype_t out_dt,
                                             float* lse, uint32_t* dev_status, qsa_stream_t stream) {
   // same checks and kernels as qsa_sparse_attn_decode; only the scratch differs
-  const size_t need = qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W);
+  const size_t need = qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv_dt);
   if (need > kScratchFloats * sizeof(float)) {
     char msg[256];
     snprintf(msg, sizeof msg,

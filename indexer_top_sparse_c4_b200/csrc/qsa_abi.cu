@@ -82,7 +82,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 1; }
+int qsa_abi_version(void) { return 2; }
 
 qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
@@ -140,9 +140,10 @@ qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, 
   return cuda_status(qsa::launch_expand_select(a, (cudaStream_t)stream), "qsa_expand_select launch");
 }
 
-size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W) {
+size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W,
+                                             qsa_dtype_t kv_dt) {
   if (T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return 0;
-  return qsa::attn_decode_ws_bytes(T, Hq, D, qsa::attn_decode_plan(T, Hkv, W).s);
+  return qsa::attn_decode_ws_bytes(T, Hq, D, qsa::attn_decode_plan(T, Hq, Hkv, D, W, kv_dt).s);
 }
 
 qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
@@ -158,7 +159,7 @@ qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void*
                                pt_stride,
                                tok, n_tok, W, T, Hq, Hkv, D, out, out_dt, k_scale, v_scale);
   if (st != QSA_OK || T == 0) return st;
-  const qsa::DecodePlan plan = qsa::attn_decode_plan(T, Hkv, W);
+  const qsa::DecodePlan plan = qsa::attn_decode_plan(T, Hq, Hkv, D, W, kv_dt);
   const size_t need = qsa::attn_decode_ws_bytes(T, Hq, D, plan.s);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
     return fail(QSA_ERR_WORKSPACE, "decode needs %zu bytes of 16-byte-aligned workspace (got %zu)",
@@ -166,7 +167,7 @@ qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void*
   qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
                   pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
                   dev_status};
-  return cuda_status(qsa::launch_sparse_attn(a, plan, workspace, (cudaStream_t)stream),
+  return cuda_status(qsa::launch_sparse_attn(a, plan, workspace, (cudaStream_t)stream, true),
                      "qsa_sparse_attn_decode launch");
 }
 
@@ -185,7 +186,8 @@ qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void
   qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
                   pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
                   dev_status};
-  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{1, 1}, nullptr, (cudaStream_t)stream),
+  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{1, 1}, nullptr, (cudaStream_t)stream,
+                                             false),
                      "qsa_sparse_attn_prefill launch");
 }
 

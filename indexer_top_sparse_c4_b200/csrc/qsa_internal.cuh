@@ -182,13 +182,21 @@ struct AttnArgs {
 // (query, KV head) merged on chip, and `s` cluster groups whose partial
 // (o, max, sum) go through the workspace to the combine kernel when s > 1.
 struct DecodePlan { int cl, s; };
-DecodePlan attn_decode_plan(int T, int Hkv, int W);
+DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
-cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s);
+// decode == true: the split plan is used; otherwise (prefill) one CTA per
+// (query, KV head) row streams all of its tokens.
+cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
+                               bool decode);
 
 // Tensor-core decode kernel (BF16 / FP8 caches, D in {128, 256}, <= 8 query
 // heads per KV head); same partial / output contract as the general kernel.
 bool attn_mma_supported(const AttnArgs& a);
+// Decode kernel on the same tensor-core tiles: one 16-token tile per warp,
+// attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on chip.
+int attn_tile_tokens();
+cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
+                                    int s, void* ws, cudaStream_t stream);
 cudaError_t launch_sparse_attn_mma(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                    int s, void* ws, cudaStream_t stream);
 

@@ -156,28 +156,86 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnArgs a, AttnSca
   }
 }
 
-// Merge the per-split partials of one (query, head): rescale every split to
-// the common maximum, add, normalise.
+// Merge the per-split partials of one (query, head): every split's weight
+// 2^(max_s - max) is computed once into shared memory, then each thread folds
+// one float4 of the output over the splits.
 template <typename OT>
 __global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs a, AttnScales sc, int splits,
                                                            const float* ws_o, const float* ws_ml) {
+  extern __shared__ __align__(16) float fs[];  // [splits] weights, then the group partials
+  __shared__ float red[8];
   pdl_wait();
   const size_t th = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const float* ml = ws_ml + th * splits * 2;
   float M = -INFINITY;
-  for (int s = 0; s < splits; ++s) M = fmaxf(M, ml[2 * s]);
+  for (int s = tid; s < splits; s += blockDim.x) M = fmaxf(M, ml[2 * s]);
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, d));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+  for (int w = 1; w < nw; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();
   float L = 0.f;
-  if (M != -INFINITY)
-    for (int s = 0; s < splits; ++s)
-      if (ml[2 * s] != -INFINITY) L = fmaf(ml[2 * s + 1], exp2f(ml[2 * s] - M), L);
-  for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
-    float O = 0.f;
-    if (L > 0.f)
-      for (int s = 0; s < splits; ++s)
-        if (ml[2 * s] != -INFINITY) O = fmaf(ws_o[(th * splits + s) * a.D + d], exp2f(ml[2 * s] - M), O);
-    store_out<OT>(reinterpret_cast<OT*>(a.out), th * a.D + d, L > 0.f ? O / L * sc.vmul : 0.f);
+  for (int s = tid; s < splits; s += blockDim.x) {
+    const float ms = ml[2 * s];
+    const float f = (M == -INFINITY || ms == -INFINITY) ? 0.f : exp2f(ms - M);
+    fs[s] = f;
+    L = fmaf(ml[2 * s + 1], f, L);
   }
-  if (threadIdx.x == 0 && a.lse) a.lse[th] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+#pragma unroll
+  for (int d = 16; d >= 1; d >>= 1) L += __shfl_xor_sync(0xffffffffu, L, d);
+  if (lane == 0) red[warp] = L;
+  __syncthreads();
+  L = 0.f;
+  for (int w = 0; w < nw; ++w) L += red[w];
+  pdl_launch_dependents();
+  __syncthreads();  // fs complete
+  const float inv = L > 0.f ? sc.vmul / L : 0.f;
+  const float* po = ws_o + th * splits * a.D;
+  // thread -> (float4 column, split group); the groups' sums meet in shared memory
+  const int ncol = a.D / 4;
+  const int ngrp = blockDim.x / ncol;  // >= 1
+  const int col = tid % ncol, grp = tid / ncol;
+  float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (grp < ngrp) {
+    int s = grp;
+    for (; s + 3 * ngrp < splits; s += 4 * ngrp) {  // four loads in flight
+      float4 v[4];
+      float f[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[u] = *reinterpret_cast<const float4*>(po + (size_t)(s + u * ngrp) * a.D + 4 * col);
+        f[u] = fs[s + u * ngrp];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        O.x = fmaf(v[u].x, f[u], O.x); O.y = fmaf(v[u].y, f[u], O.y);
+        O.z = fmaf(v[u].z, f[u], O.z); O.w = fmaf(v[u].w, f[u], O.w);
+      }
+    }
+    for (; s < splits; s += ngrp) {
+      const float4 v = *reinterpret_cast<const float4*>(po + (size_t)s * a.D + 4 * col);
+      const float f = fs[s];
+      O.x = fmaf(v.x, f, O.x); O.y = fmaf(v.y, f, O.y); O.z = fmaf(v.z, f, O.z); O.w = fmaf(v.w, f, O.w);
+    }
+  }
+  float4* part = reinterpret_cast<float4*>(fs + ((splits + 3) & ~3));  // [ngrp - 1][ncol]
+  if (grp > 0 && grp < ngrp) part[(grp - 1) * ncol + col] = O;
+  __syncthreads();
+  if (grp == 0) {
+    for (int q = 1; q < ngrp; ++q) {
+      const float4 v = part[(q - 1) * ncol + col];
+      O.x += v.x; O.y += v.y; O.z += v.z; O.w += v.w;
+    }
+    const size_t o0 = th * a.D + 4 * col;
+    store_out<OT>(reinterpret_cast<OT*>(a.out), o0, O.x * inv);
+    store_out<OT>(reinterpret_cast<OT*>(a.out), o0 + 1, O.y * inv);
+    store_out<OT>(reinterpret_cast<OT*>(a.out), o0 + 2, O.z * inv);
+    store_out<OT>(reinterpret_cast<OT*>(a.out), o0 + 3, O.w * inv);
+  }
+  if (tid == 0 && a.lse) a.lse[th] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 
 template <int D, typename QT, typename KVT, typename OT>
@@ -199,12 +257,14 @@ cudaError_t launch_combine(const AttnArgs& a, const AttnScales& sc, int splits, 
                            cudaStream_t s) {
   const float* ws_o = reinterpret_cast<const float*>(ws);
   const float* ws_ml = ws_o + (size_t)a.T * a.Hq * splits * a.D;
-  const int threads = a.D < 256 ? a.D : 256;
+  // D/4 float4 columns x 4 split groups (128 threads at D = 128, 256 at D = 256)
+  const int threads = a.D;
+  const size_t smem = ((size_t)splits + 4) * sizeof(float) + (size_t)3 * (a.D / 4) * sizeof(float4);
   if (a.out_dt == QSA_F32)
-    return launch_k(attn_combine_kernel<float>, dim3(a.T * a.Hq), dim3(threads), 0, s, 1, a, sc,
+    return launch_k(attn_combine_kernel<float>, dim3(a.T * a.Hq), dim3(threads), smem, s, 1, a, sc,
                     splits, ws_o, ws_ml);
-  return launch_k(attn_combine_kernel<__nv_bfloat16>, dim3(a.T * a.Hq), dim3(threads), 0, s, 1, a,
-                  sc, splits, ws_o, ws_ml);
+  return launch_k(attn_combine_kernel<__nv_bfloat16>, dim3(a.T * a.Hq), dim3(threads), smem, s, 1,
+                  a, sc, splits, ws_o, ws_ml);
 }
 
 template <int D, typename QT, typename KVT>
@@ -230,19 +290,27 @@ cudaError_t launch_q(const AttnArgs& a, const AttnScales& sc, int splits, void* 
 
 }  // namespace
 
-DecodePlan attn_decode_plan(int T, int Hkv, int W) {
-  // CTAs per (query, KV head): a power of two, at most 128 CTAs in all and at
-  // least one 128-token round each.  With one CTA per SM (the tensor-core
-  // kernel's shared memory) at most 33 clusters of 4 fit on the GPU at once,
-  // so clusters stay <= 4 and every cluster is resident in a single wave;
-  // cluster groups beyond that merge through the workspace.
-  const int rows = T * Hkv > 0 ? T * Hkv : 1;
-  const int tiles = (W + 15) / 16;
-  int per = 1;
-  while (per < 64 && per * 2 * rows <= 128 && per * 2 * 8 <= tiles) per <<= 1;
+DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt) {
+  AttnArgs probe{};
+  probe.kv_dt = kv_dt;
+  probe.D = D;
+  probe.Hq = Hq;
+  probe.Hkv = Hkv > 0 ? Hkv : 1;
   DecodePlan p;
-  p.cl = per < 4 ? per : 4;
-  p.s = per / p.cl;
+  if (attn_mma_supported(probe)) {
+    // tensor-core decode: one CTA per 64 token slots; every CTA's partial goes
+    // through the workspace to the combine kernel
+    p.cl = 1;
+    p.s = (W + attn_tile_tokens() - 1) / attn_tile_tokens();
+  } else {
+    // general kernel: enough splits to spread small batches over the GPU
+    const int rows = T * Hkv > 0 ? T * Hkv : 1;
+    int s = (4 * 148 + rows - 1) / rows;
+    const int max_s = (W + 63) / 64;
+    p.cl = 1;
+    p.s = s < max_s ? s : max_s;
+    if (p.s < 1) p.s = 1;
+  }
   return p;
 }
 
@@ -251,7 +319,9 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
   return (size_t)T * Hq * splits * (D + 2) * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s) {
+cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
+                               bool decode) {
+  if (!decode) plan = DecodePlan{1, 1};
   const int splits = plan.s;
   if (a.T == 0) return cudaSuccess;
   const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
@@ -261,7 +331,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   sc.vmul = fp8 ? a.v_scale : 1.f;
   cudaError_t e;
   if (attn_mma_supported(a)) {
-    e = launch_sparse_attn_mma(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
+    e = decode ? launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s)
+               : launch_sparse_attn_mma(a, sc.qk, sc.vmul, 1, 1, nullptr, s);
   } else {
     switch (a.D) {
       case 64: e = launch_q<64>(a, sc, splits, ws, s); break;

@@ -36,7 +36,8 @@ class QSAStep:
         self.out = torch.empty((T, w.Hq, w.D), dtype=out_dtype, device=dev)
         self.lse = torch.empty((T, w.Hq), dtype=torch.float32, device=dev)
         self.status = torch.zeros((1,), dtype=torch.int32, device=dev)
-        ws = 0 if self.prefill else qsa.qsa_sparse_attn_decode_workspace_size(T, w.Hq, w.Hkv, w.D, w.W)
+        ws = 0 if self.prefill else qsa.qsa_sparse_attn_decode_workspace_size(
+            T, w.Hq, w.Hkv, w.D, w.W, w.k_pages.dtype)
         self.ws_bytes = ws   # > 0: split-K partials and one combine kernel per call
         self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
         tk = qsa.qsa_topk_groups_workspace_size(T, w.K, self.score_stride)

@@ -53,7 +53,7 @@ def lib() -> ctypes.CDLL:
     L.qsa_topk_groups_workspace_size.restype = U
     L.qsa_topk_groups.argtypes = [P, I, P, I, I, P, P, P, U, P, P]
     L.qsa_expand_select.argtypes = [P, P, I, P, P, I, P, P, I, P, P]
-    L.qsa_sparse_attn_decode_workspace_size.argtypes = [I, I, I, I, I]
+    L.qsa_sparse_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
     L.qsa_sparse_attn_decode_workspace_size.restype = U
     L.qsa_sparse_attn_decode.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
                                          F, P, I, P, P, U, P, P]
@@ -138,8 +138,12 @@ def qsa_expand_select(sel, n_sel, q_pos, tok, n_tok, capture_pos=None, dev_statu
     return tok, n_tok
 
 
-def qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) -> int:
-    return int(lib().qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W))
+def qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv_dtype=QSA_FP8_E4M3) -> int:
+    """Bytes of workspace qsa_sparse_attn_decode needs; kv_dtype is a QSA_*
+    code or a torch dtype of the KV cache."""
+    if isinstance(kv_dtype, torch.dtype):
+        kv_dtype = _dt(torch.empty(0, dtype=kv_dtype))
+    return int(lib().qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv_dtype))
 
 
 def _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 1
+    assert L.qsa_abi_version() == 2
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -114,8 +114,8 @@ def test_attention_validation(L, fn):
 
 def test_decode_workspace_is_checked(L):
     # many rows (prefill-sized T) need no workspace; decode batches split across CTAs do
-    assert L.qsa_sparse_attn_decode_workspace_size(8192, 24, 2, 256, 2052) == 0
-    need = L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 2052)
+    assert L.qsa_sparse_attn_decode_workspace_size(8192, 24, 2, 256, 2052, 1) == 0
+    need = L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 2052, 1)
     assert need > 0
     ok = ctypes.c_void_p(0x10000)
     st = _attn(L, "decode", T=1, W=2052, ptr=ok, ws=ok, ws_bytes=need - 16)

@@ -188,7 +188,8 @@ def _attn_only(oracle, w, tok, n_tok, prefill, sm_scale=0.0, out_dtype=None):
     step.n_tok = torch.as_tensor(n_tok, dtype=torch.int32, device="cuda").contiguous()
     if not prefill:
         from indexer_top_sparse_c4_b200 import qsa
-        ws = qsa.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, tok.shape[1])
+        ws = qsa.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, tok.shape[1],
+                                                       w.k_pages.dtype)
         step.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device="cuda")
     w.W = tok.shape[1]
     step.attention(sm_scale=sm_scale)

@@ -39,8 +39,8 @@ def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
     for seed in (11, 12):            # two calls in a row, different inputs each time
         w = make(seed)
         step = _selection(w)
-        need = lib.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, w.W)
-        assert 0 < need <= 512 * 1024       # small batches split across CTAs: scratch in use
+        need = lib.qsa_sparse_attn_decode_workspace_size(w.T, w.Hq, w.Hkv, w.D, w.W, w.k_pages.dtype)
+        assert 0 < need <= 32 * 1024 * 1024  # per-CTA partials: scratch in use
         out = torch.full_like(step.out, float("nan"))
         lse = torch.full_like(step.lse, float("nan"))
         status = torch.zeros((1,), dtype=torch.int32, device="cuda")
@@ -57,11 +57,11 @@ def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
 
 
 def test_noalloc_refuses_shapes_beyond_its_buffer(lib):
-    # 16 queries x 16 heads x 2 split groups of 256-float partials exceed 512 KiB
-    T, Hq, Hkv, D, W = 16, 16, 1, 256, 2052
-    assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W) > 512 * 1024
+    # 64 queries x 16 heads x 129 chunk partials of 256 floats exceed 32 MiB
+    T, Hq, Hkv, D, W = 64, 16, 2, 256, 8196
+    assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, torch.uint8) > 32 * 1024 * 1024
     q = torch.zeros((T, Hq, D), dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")
+    kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")  # FP8 codes
     pt = torch.zeros((T, 1), dtype=torch.int32, device="cuda")
     tok = torch.full((T, W), -1, dtype=torch.int32, device="cuda")
     n_tok = torch.zeros((T,), dtype=torch.int32, device="cuda")
