@@ -181,7 +181,10 @@ struct AttnArgs {
 // How a decode call is spread over the GPU: clusters of `cl` CTAs per
 // (query, KV head) merged on chip, and `s` cluster groups whose partial
 // (o, max, sum) go through the workspace to the combine kernel when s > 1.
-struct DecodePlan { int cl, s; };
+struct DecodePlan {
+  int cl, s;
+  bool stream;  // tensor-core path: one CTA streams a whole row (no split)
+};
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
 // decode == true: the split plan is used; otherwise (prefill) one CTA per
@@ -195,6 +198,8 @@ bool attn_mma_supported(const AttnArgs& a);
 // Decode kernel on the same tensor-core tiles: one 16-token tile per warp,
 // attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on chip.
 int attn_tile_tokens();
+cudaError_t launch_sparse_attn_rowwarp(const AttnArgs& a, float qk_scale_log2, float vmul,
+                                       cudaStream_t stream);
 cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                     int s, void* ws, cudaStream_t stream);
 cudaError_t launch_sparse_attn_mma(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,

@@ -296,18 +296,23 @@ DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv
   probe.D = D;
   probe.Hq = Hq;
   probe.Hkv = Hkv > 0 ? Hkv : 1;
-  DecodePlan p;
+  DecodePlan p{1, 1, false};
   if (attn_mma_supported(probe)) {
-    // tensor-core decode: one CTA per 64 token slots; every CTA's partial goes
-    // through the workspace to the combine kernel
-    p.cl = 1;
-    p.s = (W + attn_tile_tokens() - 1) / attn_tile_tokens();
+    const int halves = probe.Hq / probe.Hkv > 8 ? 2 : 1;  // CTAs per KV head
+    const int ctas_per_chunk = T * probe.Hkv * halves;
+    if (ctas_per_chunk >= 148) {
+      // enough (query, KV head) rows to fill the GPU: one CTA streams each row
+      p.stream = true;
+    } else {
+      // small decode batch: one CTA per 64 token slots, partials through the
+      // workspace to the combine kernel
+      p.s = (W + attn_tile_tokens() - 1) / attn_tile_tokens();
+    }
   } else {
     // general kernel: enough splits to spread small batches over the GPU
     const int rows = T * Hkv > 0 ? T * Hkv : 1;
     int s = (4 * 148 + rows - 1) / rows;
     const int max_s = (W + 63) / 64;
-    p.cl = 1;
     p.s = s < max_s ? s : max_s;
     if (p.s < 1) p.s = 1;
   }
@@ -321,7 +326,7 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
                                bool decode) {
-  if (!decode) plan = DecodePlan{1, 1};
+  if (!decode) plan = DecodePlan{1, 1, true};
   const int splits = plan.s;
   if (a.T == 0) return cudaSuccess;
   const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
@@ -331,8 +336,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   sc.vmul = fp8 ? a.v_scale : 1.f;
   cudaError_t e;
   if (attn_mma_supported(a)) {
-    e = decode ? launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s)
-               : launch_sparse_attn_mma(a, sc.qk, sc.vmul, 1, 1, nullptr, s);
+    e = plan.stream ? launch_sparse_attn_rowwarp(a, sc.qk, sc.vmul, s)
+                    : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
   } else {
     switch (a.D) {
       case 64: e = launch_q<64>(a, sc, splits, ws, s); break;

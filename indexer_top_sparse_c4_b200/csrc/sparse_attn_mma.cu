@@ -156,11 +156,16 @@ __global__ void __launch_bounds__(Geo<FP8, D>::NW * 32) attn_mma_kernel(AttnArgs
   // then the row offsets of the current batch of token slots
   constexpr int NSTAGE = G_::NSTAGE, OFFCAP = G_::OFFCAP;
   long long* off_s = reinterpret_cast<long long*>(smem + NSTAGE * STAGE);  // [OFFCAP]
-  const int x = blockIdx.x, kvh = blockIdx.y, t = blockIdx.z;
+  const int x = blockIdx.x, t = blockIdx.z;
+  // more than 8 query heads per KV head: two CTAs, 8 heads each (the second
+  // read of the same rows hits in L2)
+  const int GQ = a.Hq / a.Hkv;
+  const int halves = GQ > 8 ? 2 : 1;
+  const int kvh = blockIdx.y / halves, half = blockIdx.y % halves;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
-  const int G = a.Hq / a.Hkv;  // <= 8
-  const int h0 = kvh * G;
+  const int G = GQ - 8 * half < 8 ? GQ - 8 * half : 8;  // this CTA's query heads
+  const int h0 = kvh * GQ + 8 * half;
 
   pdl_wait();
 
@@ -483,7 +488,7 @@ cudaError_t launch_typed(const AttnArgs& a, float qk, float vmul, int CL, int S,
   const size_t stream_bytes = (size_t)G_::NSTAGE * G_::STAGE + (size_t)G_::OFFCAP * 8;
   const size_t merge_bytes = ((size_t)G_::NW * 8 * D + G_::NW * 8 * 2 + 8 * 2) * sizeof(float);
   const size_t smem = stream_bytes > merge_bytes ? stream_bytes : merge_bytes;
-  const dim3 grid(ctas, a.Hkv, a.T);
+  const dim3 grid(ctas, a.Hkv * (a.Hq / a.Hkv > 8 ? 2 : 1), a.T);
   auto run = [&](auto kern) -> cudaError_t {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -534,11 +539,16 @@ __global__ void __launch_bounds__(kTileWarps * 32, 4) attn_tile_kernel(AttnArgs 
   __shared__ __align__(16) float wo[kTileWarps][8][D];  // per-warp O; [0] reused for the CTA
   __shared__ float wml[kTileWarps][8][2];               // per-warp (max, sum)
   __shared__ float cml[8][2];                            // CTA (max, sum)
-  const int x = blockIdx.x, kvh = blockIdx.y, t = blockIdx.z;
+  const int x = blockIdx.x, t = blockIdx.z;
+  // more than 8 query heads per KV head: two CTAs, 8 heads each (the second
+  // read of the same rows hits in L2)
+  const int GQ = a.Hq / a.Hkv;
+  const int halves = GQ > 8 ? 2 : 1;
+  const int kvh = blockIdx.y / halves, half = blockIdx.y % halves;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tq = lane & 3;
-  const int G = a.Hq / a.Hkv;  // <= 8
-  const int h0 = kvh * G;
+  const int G = GQ - 8 * half < 8 ? GQ - 8 * half : 8;  // this CTA's query heads
+  const int h0 = kvh * GQ + 8 * half;
 
   pdl_wait();
 
@@ -818,7 +828,7 @@ cudaError_t launch_tile_typed(const AttnArgs& a, float qk, float vmul, int CL, i
                               cudaStream_t s) {
   float* ws_o = reinterpret_cast<float*>(ws);
   float* ws_ml = ws_o ? ws_o + (size_t)a.T * a.Hq * S * D : nullptr;
-  const dim3 grid(CL * S, a.Hkv, a.T);
+  const dim3 grid(CL * S, a.Hkv * (a.Hq / a.Hkv > 8 ? 2 : 1), a.T);
   const dim3 block(kTileWarps * 32);
   switch (CL) {
     case 1: return launch_k(attn_tile_kernel<FP8, D, QT, OT, 1>, grid, block, 0, s, 1, a, qk, vmul, S, ws_o, ws_ml);
@@ -838,14 +848,253 @@ cudaError_t launch_tile_q(const AttnArgs& a, float qk, float vmul, int CL, int S
   return launch_tile_typed<FP8, D, float, float>(a, qk, vmul, CL, S, ws, s);
 }
 
+// ---- many rows (prefill): one warp streams one whole row --------------------
+//
+// With thousands of (query, KV head) rows there is no need to split a row: a
+// warp walks all of its row's 16-token tiles with an online softmax and writes
+// the row's output itself, so there is no merge and no workspace.  The K / V
+// tile goes straight into registers; the next tile's token -> row lookups are
+// issued before the current tile computes.  Throughput comes from the many
+// independent warps resident on every SM.
+constexpr int kRowWarps = 2;
+
+template <bool FP8, int D, typename QT, typename OT>
+__global__ void __launch_bounds__(kRowWarps * 32) attn_rowwarp_kernel(AttnArgs a, float qk_scale,
+                                                                      float vmul, int rows) {
+  using G_ = Geo<FP8, D>;
+  constexpr int CH = G_::CH, KJ = G_::KJ, KS = G_::KS, NKS = G_::NKS, VJ = G_::VJ, MT = G_::MT,
+                MTJ = G_::MTJ, ROWB = G_::ROWB;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * kRowWarps + (threadIdx.x >> 5);  // (t, KV head, head half)
+  pdl_wait();
+  if (row >= rows) return;
+  const int GQ = a.Hq / a.Hkv;
+  const int halves = GQ > 8 ? 2 : 1;
+  const int t = row / (a.Hkv * halves);
+  const int rem = row % (a.Hkv * halves);
+  const int kvh = rem / halves, half = rem % halves;
+  const int G = GQ - 8 * half < 8 ? GQ - 8 * half : 8;
+  const int h0 = kvh * GQ + 8 * half;
+  const int g = lane >> 2, tq = lane & 3;
+
+  int r = a.q_req ? a.q_req[t] : t;
+  int nt = a.n_tok[t];
+  nt = nt < 0 ? 0 : (nt > a.W ? a.W : nt);
+  if (r < 0 || r >= a.pt_rows) {
+    if (lane == 0 && kvh == 0 && half == 0) flag(a.status, QSA_DEV_BAD_REQUEST);
+    r = 0;
+    nt = 0;
+  }
+  const int32_t* trow = a.tok + (size_t)t * a.W;
+  const int32_t* pt = a.page_table + (size_t)r * a.pt_stride;
+  const size_t row_bytes = (size_t)a.Hkv * ROWB;
+  const unsigned char* kbase = reinterpret_cast<const unsigned char*>(a.k_pages);
+  const unsigned char* vbase = reinterpret_cast<const unsigned char*>(a.v_pages);
+
+  // Q^T B fragments of heads h0 + g (zero beyond G), permuted like K
+  uint32_t qb[NKS][2];
+  {
+    const QT* qrow = reinterpret_cast<const QT*>(a.q) + ((size_t)t * a.Hq + h0 + (g < G ? g : 0)) * D;
+#pragma unroll
+    for (int j = 0; j < KJ; ++j) {
+#pragma unroll
+      for (int q4 = 0; q4 < KS; ++q4) {
+        const int d0 = CH * (4 * j + tq) + 4 * q4;
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[e] = g < G ? Elem<QT>::get(qrow, d0 + e) : 0.f;
+        qb[j * KS + q4][0] = pack2<FP8>(v[0], v[1]);
+        qb[j * KS + q4][1] = pack2<FP8>(v[2], v[3]);
+      }
+    }
+  }
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  float o[MT][4];
+#pragma unroll
+  for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+
+  long long off = lane < 16 ? row_offset(a, trow, pt, lane, nt, kvh, row_bytes, ROWB) : -1;
+  for (int base = 0; base < nt; base += 16) {
+    const long long offK0 = __shfl_sync(0xffffffffu, off, g);
+    const long long offK1 = __shfl_sync(0xffffffffu, off, g + 8);
+    const long long offV0 = __shfl_sync(0xffffffffu, off, 2 * tq);
+    const long long offV1 = __shfl_sync(0xffffffffu, off, 2 * tq + 1);
+    const long long offV2 = __shfl_sync(0xffffffffu, off, 2 * tq + 8);
+    const long long offV3 = __shfl_sync(0xffffffffu, off, 2 * tq + 9);
+    const uint4 z = make_uint4(0, 0, 0, 0);
+    uint4 kr0[KJ], kr1[KJ], vr[4][VJ];
+#pragma unroll
+    for (int j = 0; j < KJ; ++j) {
+      const int cb = (4 * j + tq) * 16;
+      kr0[j] = offK0 >= 0 ? ldg16(kbase + offK0 + cb) : z;
+      kr1[j] = offK1 >= 0 ? ldg16(kbase + offK1 + cb) : z;
+    }
+#pragma unroll
+    for (int j = 0; j < VJ; ++j) {
+      const int cb = (g + 8 * j) * 16;
+      vr[0][j] = offV0 >= 0 ? ldg16(vbase + offV0 + cb) : z;
+      vr[1][j] = offV1 >= 0 ? ldg16(vbase + offV1 + cb) : z;
+      vr[2][j] = offV2 >= 0 ? ldg16(vbase + offV2 + cb) : z;
+      vr[3][j] = offV3 >= 0 ? ldg16(vbase + offV3 + cb) : z;
+    }
+    off = (lane < 16 && base + 16 < nt) ? row_offset(a, trow, pt, base + 16 + lane, nt, kvh, row_bytes, ROWB) : -1;
+
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < KJ; ++j) {
+      const uint32_t w0[4] = {kr0[j].x, kr0[j].y, kr0[j].z, kr0[j].w};
+      const uint32_t w1[4] = {kr1[j].x, kr1[j].y, kr1[j].z, kr1[j].w};
+#pragma unroll
+      for (int q4 = 0; q4 < KS; ++q4) {
+        const int ks = j * KS + q4;
+        uint32_t af[4];
+        if constexpr (FP8) {
+          af[0] = e4m3x2_to_f16x2(w0[q4]);
+          af[1] = e4m3x2_to_f16x2(w1[q4]);
+          af[2] = e4m3x2_to_f16x2(w0[q4] >> 16);
+          af[3] = e4m3x2_to_f16x2(w1[q4] >> 16);
+          if (ks & 1) mma_f16(sb, af, qb[ks][0], qb[ks][1]); else mma_f16(sa, af, qb[ks][0], qb[ks][1]);
+        } else {
+          af[0] = w0[2 * q4];
+          af[1] = w1[2 * q4];
+          af[2] = w0[2 * q4 + 1];
+          af[3] = w1[2 * q4 + 1];
+          if (ks & 1) mma_bf16(sb, af, qb[ks][0], qb[ks][1]); else mma_bf16(sa, af, qb[ks][0], qb[ks][1]);
+        }
+      }
+    }
+    const bool ok0 = offK0 >= 0, ok1 = offK1 >= 0;
+    const float s0 = ok0 ? (sa[0] + sb[0]) * qk_scale : -INFINITY;
+    const float s1 = ok0 ? (sa[1] + sb[1]) * qk_scale : -INFINITY;
+    const float s2 = ok1 ? (sa[2] + sb[2]) * qk_scale : -INFINITY;
+    const float s3 = ok1 ? (sa[3] + sb[3]) * qk_scale : -INFINITY;
+    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+#pragma unroll
+    for (int d = 4; d <= 16; d <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, d));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, d));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
+    const float al0 = exp2f(m0 - b0), al1 = exp2f(m1 - b1);
+    const float p0 = exp2f(s0 - b0), p1 = exp2f(s1 - b1), p2 = exp2f(s2 - b0), p3 = exp2f(s3 - b1);
+    m0 = mn0;
+    m1 = mn1;
+    l0 = l0 * al0 + p0 + p2;
+    l1 = l1 * al1 + p1 + p3;
+    if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        o[i][0] *= al0; o[i][1] *= al1; o[i][2] *= al0; o[i][3] *= al1;
+      }
+    }
+    const uint32_t pb0 = movmatrix_trans(pack2<FP8>(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack2<FP8>(p2, p3));
+#pragma unroll
+    for (int j = 0; j < VJ; ++j) {
+      const uint32_t va[4] = {vr[0][j].x, vr[0][j].y, vr[0][j].z, vr[0][j].w};
+      const uint32_t vb[4] = {vr[1][j].x, vr[1][j].y, vr[1][j].z, vr[1][j].w};
+      const uint32_t vc[4] = {vr[2][j].x, vr[2][j].y, vr[2][j].z, vr[2][j].w};
+      const uint32_t vd[4] = {vr[3][j].x, vr[3][j].y, vr[3][j].z, vr[3][j].w};
+#pragma unroll
+      for (int wd = 0; wd < 4; ++wd) {
+        if constexpr (FP8) {
+          const uint32_t lo01 = __byte_perm(va[wd], vb[wd], 0x5140);
+          const uint32_t hi01 = __byte_perm(va[wd], vb[wd], 0x7362);
+          const uint32_t lo89 = __byte_perm(vc[wd], vd[wd], 0x5140);
+          const uint32_t hi89 = __byte_perm(vc[wd], vd[wd], 0x7362);
+          const int mt = j * MTJ + 2 * wd;
+          uint32_t af[4];
+          af[0] = e4m3x2_to_f16x2(lo01);
+          af[1] = e4m3x2_to_f16x2(lo01 >> 16);
+          af[2] = e4m3x2_to_f16x2(lo89);
+          af[3] = e4m3x2_to_f16x2(lo89 >> 16);
+          mma_f16(o[mt], af, pb0, pb1);
+          af[0] = e4m3x2_to_f16x2(hi01);
+          af[1] = e4m3x2_to_f16x2(hi01 >> 16);
+          af[2] = e4m3x2_to_f16x2(hi89);
+          af[3] = e4m3x2_to_f16x2(hi89 >> 16);
+          mma_f16(o[mt + 1], af, pb0, pb1);
+        } else {
+          const int mt = j * MTJ + wd;
+          uint32_t af[4];
+          af[0] = __byte_perm(va[wd], vb[wd], 0x5410);
+          af[1] = __byte_perm(va[wd], vb[wd], 0x7632);
+          af[2] = __byte_perm(vc[wd], vd[wd], 0x5410);
+          af[3] = __byte_perm(vc[wd], vd[wd], 0x7632);
+          mma_bf16(o[mt], af, pb0, pb1);
+        }
+      }
+    }
+  }
+  pdl_launch_dependents();
+#pragma unroll
+  for (int d = 4; d <= 16; d <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, d);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, d);
+  }
+  // heads 2tq (c0, c2) and 2tq+1 (c1, c3); rows g / g+8 are dims d_lo / d_lo+1
+  const float inv0 = l0 > 0.f ? vmul / l0 : 0.f, inv1 = l1 > 0.f ? vmul / l1 : 0.f;
+  const size_t th0 = (size_t)t * a.Hq + h0;
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int d_lo = CH * (g + 8 * (mt / MTJ)) + 2 * (mt % MTJ);
+    if (2 * tq < G) {
+      OT* op = reinterpret_cast<OT*>(a.out) + (th0 + 2 * tq) * D + d_lo;
+      if constexpr (sizeof(OT) == 4) {
+        *reinterpret_cast<float2*>(op) = make_float2(o[mt][0] * inv0, o[mt][2] * inv0);
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[mt][0] * inv0, o[mt][2] * inv0);
+      }
+    }
+    if (2 * tq + 1 < G) {
+      OT* op = reinterpret_cast<OT*>(a.out) + (th0 + 2 * tq + 1) * D + d_lo;
+      if constexpr (sizeof(OT) == 4) {
+        *reinterpret_cast<float2*>(op) = make_float2(o[mt][1] * inv1, o[mt][3] * inv1);
+      } else {
+        *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[mt][1] * inv1, o[mt][3] * inv1);
+      }
+    }
+  }
+  if (a.lse && g == 0) {
+    if (2 * tq < G) a.lse[th0 + 2 * tq] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
+    if (2 * tq + 1 < G) a.lse[th0 + 2 * tq + 1] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
+  }
+}
+
+template <bool FP8, int D, typename QT, typename OT>
+cudaError_t launch_rowwarp_typed(const AttnArgs& a, float qk, float vmul, cudaStream_t s) {
+  const int rows = a.T * a.Hkv * (a.Hq / a.Hkv > 8 ? 2 : 1);
+  const dim3 grid((rows + kRowWarps - 1) / kRowWarps);
+  return launch_k(attn_rowwarp_kernel<FP8, D, QT, OT>, grid, dim3(kRowWarps * 32), 0, s, 1, a, qk,
+                  vmul, rows);
+}
+
+template <bool FP8, int D>
+cudaError_t launch_rowwarp_q(const AttnArgs& a, float qk, float vmul, cudaStream_t s) {
+  if (a.q_dt == QSA_BF16) {
+    if (a.out_dt == QSA_BF16) return launch_rowwarp_typed<FP8, D, __nv_bfloat16, __nv_bfloat16>(a, qk, vmul, s);
+    return launch_rowwarp_typed<FP8, D, __nv_bfloat16, float>(a, qk, vmul, s);
+  }
+  if (a.out_dt == QSA_BF16) return launch_rowwarp_typed<FP8, D, float, __nv_bfloat16>(a, qk, vmul, s);
+  return launch_rowwarp_typed<FP8, D, float, float>(a, qk, vmul, s);
+}
+
 }  // namespace
 
 bool attn_mma_supported(const AttnArgs& a) {
   return (a.kv_dt == QSA_BF16 || a.kv_dt == QSA_FP8_E4M3) && (a.D == 128 || a.D == 256) &&
-         a.Hq / a.Hkv <= 8;
+         a.Hq / a.Hkv <= 16;
 }
 
 int attn_tile_tokens() { return kTileTokens; }
+
+// Many rows: one warp streams each (query, KV head, head half) row.
+cudaError_t launch_sparse_attn_rowwarp(const AttnArgs& a, float qk, float vmul, cudaStream_t s) {
+  const bool fp8 = a.kv_dt == QSA_FP8_E4M3;
+  if (fp8) return a.D == 256 ? launch_rowwarp_q<true, 256>(a, qk, vmul, s) : launch_rowwarp_q<true, 128>(a, qk, vmul, s);
+  return a.D == 256 ? launch_rowwarp_q<false, 256>(a, qk, vmul, s) : launch_rowwarp_q<false, 128>(a, qk, vmul, s);
+}
 
 // Decode: grid (CL * S) x Hkv x T of 64-token CTAs (one tile per warp).
 cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk, float vmul, int CL, int S, void* ws,
