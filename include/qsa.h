@@ -83,6 +83,8 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
 #define QSA_DEV_ROW_RANGE 8u  /* a row's candidates exceed score_stride or
                                  its tokens exceed W */
 #define QSA_DEV_BAD_REQUEST 16u /* a request id outside [0, pt_rows) */
+#define QSA_DEV_TIMEOUT 32u   /* a bounded wait inside a kernel ran out (the
+                                 kernel stopped early; its outputs are invalid) */
 
 /* Stage 1 -- indexer scores.
  * For every query token t and complete group g < c = q_pos[t]/4 (capped at

@@ -158,6 +158,9 @@ struct IndexArgs {
   int T, H_I, D_I; float* scores; int score_stride; uint32_t* status;
 };
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t s);
+// Prefill indexer on tcgen05 (BF16 query and keys, H_I = 4, D_I = 128, T >= 32)
+bool index_tc_supported(const IndexArgs& a);
+cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s);
 
 struct TopkArgs {
   const float* scores; int score_stride; const int32_t* q_pos; int T, K;

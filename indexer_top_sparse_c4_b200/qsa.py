@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libqsa.so")
 QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = range(5)
 QSA_F32, QSA_BF16, QSA_FP8_E4M3 = 0, 1, 2
 QSA_DEV_BAD_PAGE, QSA_DEV_BAD_TOKEN, QSA_DEV_BAD_GROUP, QSA_DEV_ROW_RANGE = 1, 2, 4, 8
-QSA_DEV_BAD_REQUEST = 16
+QSA_DEV_BAD_REQUEST, QSA_DEV_TIMEOUT = 16, 32
 
 ENTRY_POINTS = (
     "qsa_index_scores", "qsa_topk_groups_workspace_size", "qsa_topk_groups",

@@ -181,7 +181,8 @@ def _add_peaks(khat, q_idx, page_table, q_req, g, device, frac=0.05, sigmas=3.0)
 
 def make(name: str, *, B: int, ctx: int, Hq: int, Hkv: int, D: int, H_I: int, D_I: int,
          K: int, kv_dtype: str, q_dtype: str, dist: str = "normal", pages: str = "perm",
-         seed: int = 0, device="cpu", q_pos=None, q_req=None, capture_pos=None) -> Workload:
+         seed: int = 0, device="cpu", q_pos=None, q_req=None, capture_pos=None,
+         idx_dtype: str = "f32") -> Workload:
     """Generic generator.  Default queries: one per request at the last token
     (decode).  Pass q_pos / q_req for prefill-style query sets."""
     g = _gen(seed, device)
@@ -197,6 +198,9 @@ def make(name: str, *, B: int, ctx: int, Hq: int, Hkv: int, D: int, H_I: int, D_
     q_idx, w_idx, khat = _indexer_inputs(T, H_I, D_I, num_pages, dist, g, device, q_req, B)
     if dist == "peaked":
         khat = _add_peaks(khat, q_idx, page_table, q_req, g, device)
+    if idx_dtype == "bf16":   # indexer query and keys stored as BF16 (RNE)
+        q_idx, _ = _store(q_idx, "bf16")
+        khat, _ = _store(khat, "bf16")
     q, _ = _store(_randn((T, Hq, D), g, device), q_dtype)
     kv_shape = (num_pages, PAGE_TOKENS, Hkv, D)
     k_pages, k_scale = _store(_randn(kv_shape, g, device), kv_dtype)
@@ -246,13 +250,14 @@ def b8_262k(K=512, device="cpu", seed=0, **kw) -> Workload:
 
 def prefill_chunk(device="cpu", seed=0, new=8192, prefix=57344, **kw) -> Workload:
     """8,192 new query tokens after a 57,344-token cached prefix (65,536 total),
-    causal, 24/2 heads of dim 256, BF16, budget 512 groups (2,048 tokens)."""
+    causal, 24/2 heads of dim 256, BF16, budget 512 groups (2,048 tokens); the
+    indexer query and keys are BF16 (the prefill scoring pass is a BF16 GEMM)."""
     ctx = prefix + new
     q_pos = torch.arange(prefix, ctx, dtype=torch.int32)
     q_req = torch.zeros(new, dtype=torch.int32)
     args = dict(B=1, ctx=ctx, Hq=24, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="bf16",
                 q_dtype="bf16", dist="normal", pages="perm", seed=seed, device=device,
-                q_pos=q_pos, q_req=q_req)
+                q_pos=q_pos, q_req=q_req, idx_dtype="bf16")
     args.update(kw)
     return make(f"prefill_{new}q_{ctx}ctx_bf16", **args)
 

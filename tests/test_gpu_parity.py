@@ -104,6 +104,28 @@ def test_prefill_chunk_sampled_rows(oracle):
     _check_step(oracle, w, step, rows=_rows(w.T, 12))
 
 
+@pytest.mark.parametrize("case", ["ragged_T", "two_requests"])
+def test_prefill_indexer_tensor_core_edges(oracle, case):
+    """The tcgen05 indexer: a query count that is not a multiple of its 32-query
+    tiles, and two requests whose boundary falls inside a tile (that tile is
+    scored on CUDA cores, the others on tensor cores)."""
+    if case == "ragged_T":
+        T, ctx = 1050, 16384
+        pos = np.sort(np.random.default_rng(1).integers(12000, ctx, T)).astype(np.int32)
+        req = np.zeros(T, np.int32)
+        B = 1
+    else:
+        T, ctx = 2048, 8192
+        pos = np.concatenate([np.arange(ctx - 1001, ctx), np.arange(ctx - 1047, ctx)]).astype(np.int32)
+        req = np.concatenate([np.zeros(1001), np.ones(1047)]).astype(np.int32)
+        B = 2
+    w = wl.make(f"tc_{case}", B=B, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=256, kv_dtype="bf16",
+                q_dtype="bf16", seed=31, device="cuda", q_pos=pos, q_req=req, idx_dtype="bf16")
+    step = QSAStep(w, prefill=True)
+    rows = sorted(set(_rows(T, 10)) | {995, 1000, 1001, 1002, 1023, 1024, 1049} & set(range(T)))
+    _check_step(oracle, w, step, rows=rows)
+
+
 def test_mtp_draft_reuse(oracle):
     w = wl.mtp(device="cuda")
     step = QSAStep(w)
