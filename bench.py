@@ -366,9 +366,83 @@ def gpu_arm(args):
     }
     if budgets:
         line["other_budgets"] = budgets
+    if args.prefill and ws == 1:
+        line["prefill"] = prefill_summary(device, stream, args.seed, 3)
     if ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.budget, args.seed, args.cpu_seconds)
     return line
+
+
+# ---- the prefill chunk ------------------------------------------------------------------
+
+def peak_bf16(sustained=False):
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops_sustained" if sustained else "bf16_tflops"]), "measured"
+    except Exception:
+        return (1400.0 if sustained else 1590.0), "fallback"
+
+
+def prefill_summary(device, stream, seed, reps):
+    """The prefill chunk (8,192 new query tokens after a 57,344-token prefix,
+    24/2 heads of dim 256, BF16 KV, budget 512 groups) through the four stages.
+    Each stage is timed alone from a CUDA graph of `reps` launches; the whole
+    step likewise.  The dense indexer contraction and the attention are
+    reported in TFLOP/s against the measured BF16 tensor peak (burst: each
+    kernel is timed on its own)."""
+    from indexer_top_sparse_c4_b200 import workloads as wl
+    from indexer_top_sparse_c4_b200.pipeline import QSAStep
+    w = wl.prefill_chunk(device=device, seed=seed)
+    st = QSAStep(w, prefill=True)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            st.run()
+        torch.cuda.synchronize()
+        times = {}
+        for name in STAGES + ("step",):
+            g = capture([st], reps, STAGES if name == "step" else (name,))
+            g.replay()
+            times[name] = replay_ms(g) / reps
+            del g
+    sum_c = int((w.q_pos // 4).sum().item())
+    sum_tok = int(st.n_tok.sum().item())
+    idx_flop = 2.0 * w.H_I * w.D_I * sum_c
+    attn_flop = 4.0 * w.D * w.Hq * sum_tok
+    peak, kind = peak_bf16()
+    idx_tf = idx_flop / (times["index_scores"] / 1e3) / 1e12
+    attn_tf = attn_flop / (times["attention"] / 1e3) / 1e12
+    names = dict(zip(STAGES, ("index_scores", "topk_groups", "expand_select", "sparse_attn_prefill")))
+    return {
+        "workload": w.name, "T": w.T, "context": int(w.q_pos.max().item()) + 1, "Hq": w.Hq, "Hkv": w.Hkv,
+        "D": w.D, "budget_groups": w.K, "kv_storage": "bf16", "indexer_operands": "bf16",
+        "query_tokens_per_s": round(w.T / (times["step"] / 1e3), 1),
+        "ms_per_step": round(times["step"], 4),
+        "stages_ms": {names[k]: round(times[k], 4) for k in STAGES},
+        "index_scores": {"bound": "tensor", "flop_per_launch": idx_flop,
+                         "achieved": round(idx_tf, 1), "peak": peak, "peak_kind": kind,
+                         "unit": "TFLOP/s", "frac": round(idx_tf / peak, 4)},
+        "sparse_attn_prefill": {"bound": "tensor", "flop_per_launch": attn_flop,
+                                "achieved": round(attn_tf, 1), "peak": peak, "peak_kind": kind,
+                                "unit": "TFLOP/s", "frac": round(attn_tf / peak, 4)},
+    }
+
+
+def prefill_arm(args):
+    """`--workload prefill`: only the prefill chunk, one JSON line."""
+    ws, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from indexer_top_sparse_c4_b200 import build
+    if not os.path.exists(build.LIB):
+        build.build()
+    stream = torch.cuda.Stream(device)
+    summary = prefill_summary(device, stream, args.seed, max(1, args.steps))
+    return {"metric": "QSA prefill query tokens/s (8,192-token chunk, 65,536 context)",
+            "value": summary["query_tokens_per_s"], "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": 3, "ms_per_step": summary["ms_per_step"],
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic", "prefill": summary}
 
 
 # ---- the oracle on host cores ----------------------------------------------------------
@@ -446,9 +520,18 @@ def main(argv=None):
     ap.add_argument("--headline-only", dest="all_budgets", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-prefill", dest="prefill", action="store_false",
+                    help="leave out the prefill-chunk summary of the decode line")
+    ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
+                    help="prefill: time only the 8,192-token prefill chunk (one GPU)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
-    line = reference_arm(args) if args.impl == "reference" else gpu_arm(args)
+    if args.impl == "reference":
+        line = reference_arm(args)
+    elif args.workload == "prefill":
+        line = prefill_arm(args)
+    else:
+        line = gpu_arm(args)
     if line is not None:
         print(json.dumps(line), flush=True)
     try:

@@ -142,8 +142,6 @@ cudaError_t launch_dims(const IndexArgs& a, cudaStream_t s) {
 
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  // many queries with BF16 operands: the tensor-core GEMM (prefill chunks)
-  if (a.T >= 1024 && index_tc_supported(a)) return launch_index_scores_tc(a, s);
   switch (a.H_I * 1000 + a.D_I) {
     case 2032: return launch_dims<2, 32>(a, s);
     case 2064: return launch_dims<2, 64>(a, s);

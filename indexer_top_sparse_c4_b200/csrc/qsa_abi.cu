@@ -103,7 +103,12 @@ qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* 
   REQUIRE(aligned16(q_idx) && aligned16(k_idx_pages), "q_idx and k_idx_pages must be 16-byte aligned");
   qsa::IndexArgs a{q_idx, q_dt, w_idx, k_idx_pages, k_dt, num_pages, page_table, pt_rows, pt_stride,
                    q_req, q_pos, T, H_I, D_I, scores, score_stride, dev_status};
-  return cuda_status(qsa::launch_index_scores(a, (cudaStream_t)stream), "qsa_index_scores launch");
+  // many queries with BF16 operands (a prefill chunk): the tensor-core GEMM;
+  // otherwise the streaming scan
+  const cudaError_t e = (T >= 256 && qsa::index_tc_supported(a))
+                            ? qsa::launch_index_scores_tc(a, (cudaStream_t)stream)
+                            : qsa::launch_index_scores(a, (cudaStream_t)stream);
+  return cuda_status(e, "qsa_index_scores launch");
 }
 
 size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride) {

@@ -19,12 +19,18 @@ from .workloads import GROUP_TOKENS, Workload
 
 
 class QSAStep:
-    def __init__(self, w: Workload, prefill: bool | None = None, out_dtype=None):
+    def __init__(self, w: Workload, prefill: bool | None = None, out_dtype=None,
+                 score_stride: int | None = None):
         self.w = w
         dev = w.q.device
         self.prefill = (w.T > 64) if prefill is None else prefill
         self.sel_pos = w.capture_pos if w.capture_pos is not None else w.q_pos
-        self.score_stride = max(1, int(self.sel_pos.max().item()) // GROUP_TOKENS)
+        if score_stride is None:
+            # the largest candidate count, rounded up to 4 so that every score
+            # row starts on 16 bytes (the tensor-core indexer then stores whole
+            # blocks of rows at once)
+            score_stride = -(-max(1, int(self.sel_pos.max().item()) // GROUP_TOKENS) // 4) * 4
+        self.score_stride = score_stride
         T = w.T
         self.scores = torch.empty((T, self.score_stride), dtype=torch.float32, device=dev)
         self.sel = torch.empty((T, w.K), dtype=torch.int32, device=dev)

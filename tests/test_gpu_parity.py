@@ -104,26 +104,73 @@ def test_prefill_chunk_sampled_rows(oracle):
     _check_step(oracle, w, step, rows=_rows(w.T, 12))
 
 
-@pytest.mark.parametrize("case", ["ragged_T", "two_requests"])
+@pytest.mark.parametrize("case", ["ragged_T", "two_requests", "many_runs_odd_stride"])
 def test_prefill_indexer_tensor_core_edges(oracle, case):
-    """The tcgen05 indexer: a query count that is not a multiple of its 32-query
-    tiles, and two requests whose boundary falls inside a tile (that tile is
-    scored on CUDA cores, the others on tensor cores)."""
+    """The tcgen05 indexer: a query count that is not a multiple of its
+    128-query tiles; request boundaries inside a tile (each run of one
+    request's queries gets its own pass, and blocks shared by two runs are
+    written row by row); a score stride that is not a multiple of 4 (rows not
+    16-byte aligned, so no block store at all)."""
+    stride = None
     if case == "ragged_T":
         T, ctx = 1050, 16384
         pos = np.sort(np.random.default_rng(1).integers(12000, ctx, T)).astype(np.int32)
         req = np.zeros(T, np.int32)
         B = 1
-    else:
+    elif case == "two_requests":
         T, ctx = 2048, 8192
         pos = np.concatenate([np.arange(ctx - 1001, ctx), np.arange(ctx - 1047, ctx)]).astype(np.int32)
         req = np.concatenate([np.zeros(1001), np.ones(1047)]).astype(np.int32)
         B = 2
+    else:
+        T, ctx = 300, 4096
+        sizes = [37, 1, 90, 59, 113]   # boundaries at 37, 38, 128, 187 inside the first three tiles
+        req = np.concatenate([np.full(n, r % 3) for r, n in enumerate(sizes)]).astype(np.int32)
+        pos = np.concatenate([np.sort(np.random.default_rng(n).integers(300, ctx, n)) for n in sizes])
+        pos = pos.astype(np.int32)
+        B = 3
+        stride = ctx // 4 + 3
     w = wl.make(f"tc_{case}", B=B, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=256, kv_dtype="bf16",
                 q_dtype="bf16", seed=31, device="cuda", q_pos=pos, q_req=req, idx_dtype="bf16")
-    step = QSAStep(w, prefill=True)
-    rows = sorted(set(_rows(T, 10)) | {995, 1000, 1001, 1002, 1023, 1024, 1049} & set(range(T)))
+    step = QSAStep(w, prefill=True, score_stride=stride)
+    boundaries = {0, 36, 37, 38, 127, 128, 186, 187, 299, 995, 1000, 1001, 1002, 1023, 1024, 1049}
+    rows = sorted(set(_rows(T, 10)) | (boundaries & set(range(T))))
     _check_step(oracle, w, step, rows=rows)
+
+
+def test_prefill_indexer_bad_request_rows():
+    """Rows whose request id is outside the page table get -inf for every
+    candidate and raise QSA_DEV_BAD_REQUEST; the rows around them, in the same
+    128-query tiles, still score correctly."""
+    from indexer_top_sparse_c4_b200 import qsa
+    T, ctx = 384, 8192
+    pos = np.sort(np.random.default_rng(5).integers(2000, ctx, T)).astype(np.int32)
+    w = wl.make("tc_bad_req", B=1, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=256, kv_dtype="bf16",
+                q_dtype="bf16", seed=9, device="cuda", q_pos=pos, q_req=np.zeros(T, np.int32),
+                idx_dtype="bf16")
+    w.q_req[200:261] = 7   # the page table has one row
+    step = QSAStep(w, prefill=True)
+    step.index_scores()
+    torch.cuda.synchronize()
+    st = int(step.status.item())
+    assert st & qsa.QSA_DEV_BAD_REQUEST and not st & qsa.QSA_DEV_TIMEOUT
+    scores = host(step.scores)
+    for t in range(200, 261):
+        assert np.all(np.isneginf(scores[t, : pos[t] // 4]))
+    good = [0, 127, 128, 199, 261, 300, 383]
+    n = {k: host(getattr(w, k)) for k in ("q_idx", "w_idx", "k_idx_pages", "page_table", "q_req", "q_pos")}
+    ref, _ = oracle_scores(n, good, step.score_stride)
+    bound = score_bound(n["q_idx"], n["w_idx"], n["k_idx_pages"], n["page_table"], n["q_req"], n["q_pos"],
+                        good, step.score_stride)
+    for i, t in enumerate(good):
+        c = pos[t] // 4
+        assert np.all(np.abs(scores[t, :c].astype(np.float64) - ref[i, :c]) <= bound[i, :c] + 1e-30)
+
+
+def oracle_scores(n, rows, stride):
+    import oracle as orc
+    return orc.index_scores(n["q_idx"][rows], n["w_idx"][rows], n["k_idx_pages"], n["page_table"],
+                            n["q_pos"][rows], n["q_req"][rows], stride)
 
 
 def test_mtp_draft_reuse(oracle):
