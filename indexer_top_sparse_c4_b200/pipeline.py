@@ -27,8 +27,7 @@ class QSAStep:
         self.sel_pos = w.capture_pos if w.capture_pos is not None else w.q_pos
         if score_stride is None:
             # the largest candidate count, rounded up to 4 so that every score
-            # row starts on 16 bytes (the tensor-core indexer then stores whole
-            # blocks of rows at once)
+            # row starts on 16 bytes
             score_stride = -(-max(1, int(self.sel_pos.max().item()) // GROUP_TOKENS) // 4) * 4
         self.score_stride = score_stride
         T = w.T
