@@ -191,7 +191,7 @@ qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void
   qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
                   pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
                   dev_status};
-  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{1, 1, true}, nullptr, (cudaStream_t)stream,
+  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{1, 1, true, false}, nullptr, (cudaStream_t)stream,
                                              false),
                      "qsa_sparse_attn_prefill launch");
 }

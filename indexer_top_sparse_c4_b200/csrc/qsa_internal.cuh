@@ -186,7 +186,8 @@ struct AttnArgs {
 // (o, max, sum) go through the workspace to the combine kernel when s > 1.
 struct DecodePlan {
   int cl, s;
-  bool stream;  // tensor-core path: one CTA streams a whole row (no split)
+  bool stream;   // tensor-core path: one CTA streams a whole row (no split)
+  bool cluster;  // tensor-core path: one cluster of cl CTAs per row, merged on chip
 };
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
@@ -198,6 +199,12 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
 // Tensor-core decode kernel (BF16 / FP8 caches, D in {128, 256}, <= 8 query
 // heads per KV head); same partial / output contract as the general kernel.
 bool attn_mma_supported(const AttnArgs& a);
+// Decode kernel with one thread-block cluster of cl CTAs per (query, KV head)
+// row: no workspace, no combine.  Token slots one pass of the kernel covers
+// per warp step (larger rows take several steps).
+int attn_cluster_tokens_per_round(qsa_dtype_t kv_dt, int D, int cl);
+cudaError_t launch_sparse_attn_cluster(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
+                                       cudaStream_t s);
 // Decode kernel on the same tensor-core tiles: one 16-token tile per warp,
 // attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on chip.
 int attn_tile_tokens();

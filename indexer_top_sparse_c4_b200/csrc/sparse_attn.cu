@@ -296,13 +296,21 @@ DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv
   probe.D = D;
   probe.Hq = Hq;
   probe.Hkv = Hkv > 0 ? Hkv : 1;
-  DecodePlan p{1, 1, false};
+  DecodePlan p{1, 1, false, false};
   if (attn_mma_supported(probe)) {
     const int halves = probe.Hq / probe.Hkv > 8 ? 2 : 1;  // CTAs per KV head
     const int ctas_per_chunk = T * probe.Hkv * halves;
+    int cl = 8;  // the largest cluster that keeps every row's cluster resident at once
+    while (cl > 1 && ctas_per_chunk * cl > 148) cl >>= 1;
+    const int rounds = (W + attn_cluster_tokens_per_round(kv_dt, D, cl) - 1) /
+                       attn_cluster_tokens_per_round(kv_dt, D, cl);
     if (ctas_per_chunk >= 148) {
       // enough (query, KV head) rows to fill the GPU: one CTA streams each row
       p.stream = true;
+    } else if (rounds <= 3) {
+      // a cluster covers a whole row in at most three steps per warp
+      p.cluster = true;
+      p.cl = cl;
     } else {
       // small decode batch: one CTA per 64 token slots, partials through the
       // workspace to the combine kernel
@@ -326,7 +334,7 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
                                bool decode) {
-  if (!decode) plan = DecodePlan{1, 1, true};
+  if (!decode) plan = DecodePlan{1, 1, true, false};
   const int splits = plan.s;
   if (a.T == 0) return cudaSuccess;
   const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
@@ -336,8 +344,9 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   sc.vmul = fp8 ? a.v_scale : 1.f;
   cudaError_t e;
   if (attn_mma_supported(a)) {
-    e = plan.stream ? launch_sparse_attn_rowwarp(a, sc.qk, sc.vmul, s)
-                    : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
+    e = plan.stream    ? launch_sparse_attn_rowwarp(a, sc.qk, sc.vmul, s)
+        : plan.cluster ? launch_sparse_attn_cluster(a, sc.qk, sc.vmul, plan.cl, s)
+                       : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
   } else {
     switch (a.D) {
       case 64: e = launch_q<64>(a, sc, splits, ws, s); break;

@@ -36,106 +36,14 @@
 
 #include <cooperative_groups.h>
 
-#include "qsa_internal.cuh"
+#include "attn_common.cuh"
 
 namespace cg = cooperative_groups;
 
 namespace qsa {
 namespace {
 
-constexpr float kLn2 = 0.69314718055994530942f;
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
-  uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(y) : "r"(x));
-  return y;
-}
-
-// two FP8-E4M3 codes (low byte first) -> f16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
-template <bool FP8> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
-template <> __device__ __forceinline__ uint32_t pack2<true>(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-template <> __device__ __forceinline__ uint32_t pack2<false>(float lo, float hi) {
-  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_addr), "l"(gptr) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
-
-// Tile geometry for one KV storage type and head dim.
-template <bool FP8, int D>
-struct Geo {
-  static constexpr int EB = FP8 ? 1 : 2;       // bytes per element
-  static constexpr int CH = 16 / EB;           // elements per 16-byte chunk
-  static constexpr int NCH = D / CH;           // chunks per row
-  static constexpr int KJ = NCH / 4;           // K chunks per thread per row
-  static constexpr int KS = CH / 4;            // k-steps per chunk
-  static constexpr int NKS = D / 16;           // k-steps per row
-  static constexpr int VJ = NCH / 8;           // V chunks per thread per token
-  static constexpr int MT = D / 16;            // PV m-tiles (output dims / 16)
-  static constexpr int MTJ = CH / 2;           // m-tiles fed by one V chunk
-  static constexpr int ROWB = D * EB;          // bytes of one K (or V) row of one KV head
-  static constexpr int NW = 4;                 // warps per CTA: a round is one tile per warp
-  static constexpr int ROUND = 16 * NW;        // tokens per round
-  static constexpr int STAGE = ROUND * 2 * ROWB;  // K rows, then V rows
-  // FP8 rows are half the size: three 32 KiB stages keep a CTA near 104 KiB of
-  // shared memory, two CTAs per SM, so clusters of 8 all fit at once; BF16
-  // keeps two 64 KiB stages at one CTA per SM
-  static constexpr int NSTAGE = FP8 ? 3 : 2;
-  static constexpr int OFFCAP = 1024;          // row offsets looked up per batch
-  static_assert(NCH % 8 == 0, "V chunks must split over 8 lanes");
-  static_assert(OFFCAP % ROUND == 0, "a batch holds whole rounds");
-};
-
-// Byte offset of the K/V row (this KV head) of token slot `i` of the list, or
-// -1 for padding, a slot past `end`, or an id / page outside the cache.
-__device__ __forceinline__ long long row_offset(const AttnArgs& a, const int32_t* trow,
-                                                const int32_t* pt, int i, int end, int kvh,
-                                                size_t row_bytes, size_t head_bytes) {
-  if (i >= end) return -1;
-  const int j = __ldg(trow + i);
-  if (j == -1) return -1;
-  if (j < -1 || j / kPageTokens >= a.pt_stride) {
-    flag(a.status, QSA_DEV_BAD_TOKEN);
-    return -1;
-  }
-  const int page = __ldg(pt + j / kPageTokens);
-  if (page < 0 || page >= a.num_pages) {
-    flag(a.status, QSA_DEV_BAD_PAGE);
-    return -1;
-  }
-  return (long long)(((size_t)page * kPageTokens + (j % kPageTokens)) * row_bytes + (size_t)kvh * head_bytes);
-}
+using namespace attn;
 
 // grid (CL * S, Hkv, T), clusters of CL CTAs along x, NW warps per CTA.  CTA
 // x covers token slots [x * chunk, (x + 1) * chunk) of its (query, KV head) in

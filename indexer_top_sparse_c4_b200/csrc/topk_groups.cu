@@ -5,17 +5,23 @@
 //
 // Design (sm_100a): one thread-block cluster of CL CTAs x 512 threads per
 // query row; thread i of CTA r owns KPT consecutive candidates in registers as
-// order-preserving uint32 keys, so the row is read from memory once.
+// order-preserving uint32 keys, so the row is read from memory once (16-byte
+// loads where the row is aligned).
 //  * Radix select, 8 bits per pass from the most significant end, finds the
 //    exact key tau of the n-th largest candidate.  Each pass histograms only
 //    the keys that still match the digits found so far: per-warp shared
-//    histograms (no block-wide atomic hot spots), one block reduction, and one
-//    distributed-shared-memory add into CTA 0's histogram for the cluster.
+//    histograms (no block-wide atomic hot spots), one block reduction, and
+//    then every CTA WRITES its 256 counts into its own slot of that pass's
+//    table in every CTA of the cluster.  After one cluster barrier each CTA
+//    adds the CL slots locally and finds the digit itself: one barrier per
+//    pass, no remote reads, no zeroing.
 //  * Output: every key > tau is kept, plus the first `need` keys == tau in
 //    index order.  Because each thread owns a contiguous run of ids, one
-//    exclusive scan over threads and one over the cluster's CTAs give every
-//    thread the position of its first kept id: the ids come out ascending with
-//    no sort.
+//    exclusive scan over threads gives every thread the position of its first
+//    kept id within its CTA; the counts of the CTAs before it come from the
+//    histogram tables every CTA already holds (keys above tau are the keys
+//    above the chosen digit in some pass), so no further exchange is needed
+//    and the ids come out ascending with no sort.
 #include <cooperative_groups.h>
 
 #include "qsa_internal.cuh"
@@ -28,13 +34,14 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
+constexpr int kMaxCL = 8;
 
 struct TopkSmem {
-  uint32_t hw[kWarps][kBins];  // per-warp histogram of the current digit
-  uint32_t ghist[4][kBins];    // cluster histogram per pass (CTA 0's copy is used)
-  int cnt_gt[8], cnt_eq[8];    // per-CTA counts of keys > tau and == tau
-  int wa[kWarps], wb[kWarps];  // per-warp scan totals
-  int bin, above;
+  uint32_t hw[kWarps][kBins];            // per-warp histogram of the current digit
+  uint32_t hall[4][kMaxCL][kBins];       // per pass: slot q = CTA q's histogram
+  int wsum[kWarps][kMaxCL];              // block reduction of the per-CTA counts above tau
+  int wa[kWarps];                        // per-warp scan totals
+  int bin[4], above;
 };
 
 // float -> uint32 whose unsigned order equals the float order; -0 maps like +0.
@@ -74,7 +81,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 }
 
 template <int CL, int KPT>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -103,13 +110,19 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
   const float* row = a.scores + (size_t)t * a.score_stride;
   uint32_t keys[KPT];
 #pragma unroll
-  for (int j = 0; j < KPT; ++j) keys[j] = first + j < c ? order_key(__ldg(row + first + j)) : 0u;
-  for (int i = tid; i < 4 * kBins; i += kThreads) (&sm.ghist[0][0])[i] = 0u;
+  for (int j = 0; j < KPT; j += 4) {
+    if (vec && first + j + 3 < c) {  // 16-byte aligned when the row stride is a multiple of 4
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + first + j));
+      keys[j] = order_key(v.x);
+      keys[j + 1] = order_key(v.y);
+      keys[j + 2] = order_key(v.z);
+      keys[j + 3] = order_key(v.w);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) keys[j + e] = first + j + e < c ? order_key(__ldg(row + first + j + e)) : 0u;
+    }
+  }
   pdl_launch_dependents();
-  csync<CL>();  // every CTA's cluster histograms are zero before anyone adds
-
-  uint32_t* ghist0 = &sm.ghist[0][0];
-  if constexpr (CL > 1) ghist0 = cg::this_cluster().map_shared_rank(ghist0, 0);
 
   // ---- radix select: 4 passes of 8 bits locate tau
   uint32_t prefix = 0;
@@ -132,16 +145,20 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) v += sm.hw[w][tid];
       if constexpr (CL > 1) {
-        if (v) atomicAdd(ghist0 + pass * kBins + tid, v);
+        cg::cluster_group cl = cg::this_cluster();
+#pragma unroll
+        for (int q = 0; q < CL; ++q) cl.map_shared_rank(&sm.hall[pass][rank][tid], q)[0] = v;
       } else {
-        sm.ghist[pass][tid] = v;
+        sm.hall[pass][0][tid] = v;
       }
     }
-    csync<CL>();
+    csync<CL>();  // every CTA's counts are in every CTA's table
     // the bin holding the need-th largest: thread i looks at bin 255 - i, so
     // an exclusive scan over threads counts the keys in all higher bins
     if (tid < kBins) {
-      const int h = (int)ghist0[pass * kBins + (kBins - 1 - tid)];
+      int h = 0;
+#pragma unroll
+      for (int q = 0; q < CL; ++q) h += (int)sm.hall[pass][q][kBins - 1 - tid];
       int incl = h;
 #pragma unroll
       for (int d = 1; d < 32; d <<= 1) {
@@ -153,16 +170,38 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
       int above = incl - h;
       for (int w = 0; w < warp; ++w) above += sm.wa[w];
       if (above < need && above + h >= need) {
-        sm.bin = kBins - 1 - tid;
+        sm.bin[pass] = kBins - 1 - tid;
         sm.above = above;
       }
     }
     __syncthreads();
-    prefix |= (uint32_t)sm.bin << shift;
+    prefix |= (uint32_t)sm.bin[pass] << shift;
     need -= sm.above;
     __syncthreads();
   }
   const uint32_t tau = prefix;
+
+  // ---- keys above tau in each CTA: a key is above tau when, in the first
+  // pass where its digit differs from tau's, its digit is the larger one, and
+  // that pass's table counted it under that digit in its CTA's slot
+  if (tid < kBins) {
+    int x[kMaxCL];
+#pragma unroll
+    for (int q = 0; q < CL; ++q) x[q] = 0;
+#pragma unroll
+    for (int pass = 0; pass < 4; ++pass) {
+      if (tid > sm.bin[pass]) {
+#pragma unroll
+        for (int q = 0; q < CL; ++q) x[q] += (int)sm.hall[pass][q][tid];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < CL; ++q) {
+#pragma unroll
+      for (int d = 16; d >= 1; d >>= 1) x[q] += __shfl_xor_sync(0xffffffffu, x[q], d);
+      if (lane == 0) sm.wsum[warp][q] = x[q];
+    }
+  }
 
   // ---- kept ids: all keys > tau, then the first `need` keys == tau by id
   int gt = 0, eq = 0;
@@ -171,27 +210,18 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a) {
     gt += keys[j] > tau;
     eq += keys[j] == tau;
   }
-  int gt_cta, eq_cta;
-  const int gt_before = block_exclusive_scan(gt, sm.wa, gt_cta);
-  const int eq_before = block_exclusive_scan(eq, sm.wb, eq_cta);
-  if (tid == 0) {
-    if constexpr (CL > 1) {
-      cg::cluster_group cl = cg::this_cluster();
-      for (int q = 0; q < CL; ++q) {
-        cl.map_shared_rank(sm.cnt_gt, q)[rank] = gt_cta;
-        cl.map_shared_rank(sm.cnt_eq, q)[rank] = eq_cta;
-      }
-    } else {
-      sm.cnt_gt[0] = gt_cta;
-      sm.cnt_eq[0] = eq_cta;
-    }
-  }
-  csync<CL>();  // last cluster-wide step: from here every access is local
+  int both;  // one scan of gt (low 16 bits) and eq (high): per-CTA counts stay below 2^16
+  const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum visible
+  const int gt_before = before & 0xffff, eq_before = before >> 16;
   int off = 0, eq_prev = 0;
   for (int q = 0; q < rank; ++q) {
+    int gt_q = 0;
+#pragma unroll
+    for (int w = 0; w < kBins / 32; ++w) gt_q += sm.wsum[w][q];
+    const int eq_q = (int)sm.hall[3][q][sm.bin[3]];
     const int rem = need - eq_prev;
-    off += sm.cnt_gt[q] + (rem <= 0 ? 0 : (rem < sm.cnt_eq[q] ? rem : sm.cnt_eq[q]));
-    eq_prev += sm.cnt_eq[q];
+    off += gt_q + (rem <= 0 ? 0 : (rem < eq_q ? rem : eq_q));
+    eq_prev += eq_q;
   }
   int rem = need - eq_prev;                     // tau-keys still to take at this CTA's start
   rem = rem < 0 ? 0 : rem;
@@ -223,7 +253,8 @@ cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
   auto kern = topk_kernel<CL, KPT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a);
+  const int vec = (a.score_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
+  return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec);
 }
 
 template <int KPT>

@@ -113,12 +113,14 @@ def test_attention_validation(L, fn):
 
 
 def test_decode_workspace_is_checked(L):
-    # many rows (prefill-sized T) need no workspace; decode batches split across CTAs do
+    # many rows (prefill-sized T) and rows one cluster covers need no
+    # workspace; rows split across cluster groups do
     assert L.qsa_sparse_attn_decode_workspace_size(8192, 24, 2, 256, 2052, 1) == 0
-    need = L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 2052, 1)
+    assert L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 2052, 1) == 0
+    need = L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 8196, 1)
     assert need > 0
     ok = ctypes.c_void_p(0x10000)
-    st = _attn(L, "decode", T=1, W=2052, ptr=ok, ws=ok, ws_bytes=need - 16)
+    st = _attn(L, "decode", T=1, W=8196, ptr=ok, ws=ok, ws_bytes=need - 16)
     assert st == 3 and str(need) in _err(L)
 
 

@@ -31,11 +31,13 @@ def _selection(w):
     return step
 
 
-@pytest.mark.parametrize("which", ["b1_16k_bf16", "b2_16k_fp8"])
+@pytest.mark.parametrize("which", ["b1_16k_bf16_k2048", "b2_16k_fp8_k4096"])
 def test_noalloc_matches_workspace_decode_on_two_calls(lib, which):
+    # rows too long for one cluster (8,196 BF16 / 16,388 FP8 token slots) are
+    # split over CTA groups whose partials go through the scratch buffer
     from indexer_top_sparse_c4_b200 import workloads as wl
-    make = (lambda s: wl.b1_16k(device="cuda", seed=s)) if which == "b1_16k_bf16" else \
-        (lambda s: wl.b1_16k(device="cuda", seed=s, B=2, kv_dtype="fp8"))
+    make = (lambda s: wl.b1_16k(device="cuda", seed=s, K=2048)) if which == "b1_16k_bf16_k2048" else \
+        (lambda s: wl.b1_16k(device="cuda", seed=s, B=2, kv_dtype="fp8", K=4096))
     for seed in (11, 12):            # two calls in a row, different inputs each time
         w = make(seed)
         step = _selection(w)
