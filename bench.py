@@ -1,7 +1,8 @@
 """Benchmark of the QSA decode hot path on B200: B8 x 262,144-token FP8 KV.
 
 One step = one layer's decode of 8 requests through all four stages of
-libqsa.so (indexer scores -> Top-K groups -> expand -> sparse attention),
+libqsa.so in three launches (indexer scores -> Top-K groups expanded to tokens ->
+sparse attention),
 inputs resident in HBM.  Prints ONE JSON line (rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--budget 512]
@@ -33,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QSA sparse-decode tokens/s @B8×262K FP8 KV; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
-KERNELS_PER_STEP = 4  # index, topk, expand, attention (partials merged inside the attention clusters)
+KERNELS_PER_STEP = 3  # index, Top-K with expansion, attention (partials merged inside the clusters)
 
 
 def peak_hbm():
@@ -174,8 +175,8 @@ def make_sets(K, device, seed, n_sets=2, context=262144):
     return sets
 
 
-STAGES = ("index_scores", "topk", "expand", "attention")
-STAGE_NAMES = ("index_scores", "topk_groups", "expand_select", "sparse_attn_decode")
+STAGES = ("index_scores", "select", "attention")
+STAGE_NAMES = ("index_scores", "topk_expand", "sparse_attn_decode")
 
 
 def capture(sets, steps, stages=STAGES):
@@ -413,7 +414,7 @@ def prefill_summary(device, stream, seed, reps):
     peak, kind = peak_bf16()
     idx_tf = idx_flop / (times["index_scores"] / 1e3) / 1e12
     attn_tf = attn_flop / (times["attention"] / 1e3) / 1e12
-    names = dict(zip(STAGES, ("index_scores", "topk_groups", "expand_select", "sparse_attn_prefill")))
+    names = dict(zip(STAGES, ("index_scores", "topk_expand", "sparse_attn_prefill")))
     return {
         "workload": w.name, "T": w.T, "context": int(w.q_pos.max().item()) + 1, "Hq": w.Hq, "Hkv": w.Hkv,
         "D": w.D, "budget_groups": w.K, "kv_storage": "bf16", "indexer_operands": "bf16",

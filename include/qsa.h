@@ -131,6 +131,16 @@ QSA_API qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel,
                                int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
                                qsa_stream_t stream);
 
+/* Stages 2 and 3 in one launch, for rows without an MTP capture: exactly
+ * qsa_topk_groups(scores, score_stride, q_pos, T, K, sel, n_sel) followed by
+ * qsa_expand_select(sel, n_sel, K, q_pos, NULL, T, tok, n_tok, W), with the
+ * same outputs, layouts and status bits.  The expansion is not defined by
+ * the pages as a separate pass: joining it to the selection saves a launch
+ * and a read of sel on the decode path.  W >= 4*K + 4. */
+QSA_API qsa_status_t qsa_topk_expand(const float* scores, int score_stride, const int32_t* q_pos, int T,
+                             int K, int32_t* sel, int32_t* n_sel, int32_t* tok, int32_t* n_tok,
+                             int W, uint32_t* dev_status, qsa_stream_t stream);
+
 /* Stage 4 -- GQA attention over the selected tokens ("QSA in brief": only the
  * selected entries are read; the Ascend article: rows with nothing to attend
  * give exact zeros, the D-based scale is the default).
@@ -200,8 +210,8 @@ QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
 QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */
 QSA_API const char* qsa_status_name(qsa_status_t s);
-/* ABI version: bumped on any signature change (2: the decode workspace query
- * takes the KV dtype). */
+/* ABI version: bumped on any change of the entry points (2: the decode
+ * workspace query takes the KV dtype; 3: qsa_topk_expand). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

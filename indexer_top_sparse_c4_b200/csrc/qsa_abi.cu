@@ -82,7 +82,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 2; }
+int qsa_abi_version(void) { return 3; }
 
 qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
@@ -143,6 +143,22 @@ qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, 
   REQUIRE(sel && n_sel && q_pos && tok && n_tok, "null pointer argument");
   qsa::ExpandArgs a{sel, n_sel, K, q_pos, capture_pos, T, tok, n_tok, W, dev_status};
   return cuda_status(qsa::launch_expand_select(a, (cudaStream_t)stream), "qsa_expand_select launch");
+}
+
+qsa_status_t qsa_topk_expand(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,
+                             int32_t* sel, int32_t* n_sel, int32_t* tok, int32_t* n_tok, int W,
+                             uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
+  REQUIRE(W >= 4 * K + 4, "W must be >= 4*K + 4 = %d (got %d)", 4 * K + 4, W);
+  REQUIRE(score_stride >= 1, "score_stride must be >= 1");
+  SUPPORT(qsa::topk_cluster_size(score_stride) > 0, "score_stride %d exceeds the %d groups a row may hold",
+          score_stride, 8 * 49152);
+  if (T == 0) return QSA_OK;
+  REQUIRE(scores && q_pos && sel && n_sel && tok && n_tok, "null pointer argument");
+  qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status, tok, n_tok, W};
+  return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_expand launch");
 }
 
 size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W,

@@ -165,6 +165,9 @@ cudaError_t launch_index_scores_tc(const IndexArgs& a, cudaStream_t s);
 struct TopkArgs {
   const float* scores; int score_stride; const int32_t* q_pos; int T, K;
   int32_t* sel; int32_t* n_sel; uint32_t* status;
+  // optional: also expand the kept groups to token ids (no MTP capture);
+  // tok == nullptr skips it
+  int32_t* tok = nullptr; int32_t* n_tok = nullptr; int W = 0;
 };
 int topk_cluster_size(int score_stride);       // 0: unsupported
 cudaError_t launch_topk_groups(const TopkArgs& a, cudaStream_t s);

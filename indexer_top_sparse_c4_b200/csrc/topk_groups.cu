@@ -81,7 +81,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 }
 
 template <int CL, int KPT>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec) {
+__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int tvec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -98,9 +98,22 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec) {
   const int K = a.K;
   const int n = c < K ? c : K;
   int32_t* out = a.sel + (size_t)t * K;
+  // the expanded row (when asked for): 4 tokens per kept group, then the
+  // current block 4*c(p) .. p, then -1
+  int32_t* trow = a.tok ? a.tok + (size_t)t * a.W : nullptr;
+  const int cb = p >= 0 ? p - kGroupTokens * (p / kGroupTokens) + 1 : 0;  // current-block tokens
   if (c <= K) {  // every candidate is kept: dense fallback (uniform over the cluster)
     pdl_launch_dependents();
     for (int i = rank * kThreads + tid; i < K; i += CL * kThreads) out[i] = i < c ? i : -1;
+    if (trow) {  // tokens 0 .. p (the kept groups and the current block are contiguous)
+      const int total = kGroupTokens * n + cb;
+      for (int i = rank * kThreads + tid; i < a.W; i += CL * kThreads)
+        trow[i] = i < total ? (i < kGroupTokens * n ? i : kGroupTokens * (p / kGroupTokens) + i - kGroupTokens * n) : -1;
+      if (rank == 0 && tid == 0) {
+        a.n_tok[t] = total < a.W ? total : a.W;
+        if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
+      }
+    }
     if (rank == 0 && tid == 0) a.n_sel[t] = n;
     return;
   }
@@ -237,13 +250,34 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec) {
       --take;
     }
     if (keep) {
-      if (pos < K) out[pos] = first + j;
+      if (pos < K) {
+        const int g = first + j;
+        out[pos] = g;
+        if (trow) {
+          if (tvec) {
+            *reinterpret_cast<int4*>(trow + kGroupTokens * pos) =
+                make_int4(kGroupTokens * g, kGroupTokens * g + 1, kGroupTokens * g + 2, kGroupTokens * g + 3);
+          } else {
+#pragma unroll
+            for (int e = 0; e < kGroupTokens; ++e) trow[kGroupTokens * pos + e] = kGroupTokens * g + e;
+          }
+        }
+      }
       ++pos;
     }
   }
   if (rank == 0) {
     for (int i = n + tid; i < K; i += kThreads) out[i] = -1;
     if (tid == 0) a.n_sel[t] = n;
+    if (trow) {  // the current block, then padding
+      const int head = kGroupTokens * n, total = head + cb;
+      for (int i = head + tid; i < a.W; i += kThreads)
+        trow[i] = i < total ? kGroupTokens * (p / kGroupTokens) + (i - head) : -1;
+      if (tid == 0) {
+        a.n_tok[t] = total < a.W ? total : a.W;
+        if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
+      }
+    }
   }
 }
 
@@ -254,7 +288,8 @@ cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int vec = (a.score_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
-  return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec);
+  const int tvec = a.tok && a.W % 4 == 0 && (reinterpret_cast<uintptr_t>(a.tok) & 15u) == 0;
+  return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec, tvec);
 }
 
 template <int KPT>

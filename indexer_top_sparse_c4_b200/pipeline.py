@@ -74,9 +74,18 @@ class QSAStep:
             qsa.qsa_sparse_attn_decode(w.q, w.k_pages, w.v_pages, w.page_table, self.tok,
                                        self.n_tok, self.out, workspace=self.ws, **common)
 
+    def select(self, stream=None):
+        """Top-K and expansion: one launch when there is no MTP capture."""
+        w = self.w
+        if w.capture_pos is None:
+            qsa.qsa_topk_expand(self.scores, w.q_pos, w.K, self.sel, self.n_sel, self.tok, self.n_tok,
+                                dev_status=self.status, stream=stream)
+        else:
+            self.topk(stream)
+            self.expand(stream)
+
     def run(self, stream=None, sm_scale=0.0):
         self.index_scores(stream)
-        self.topk(stream)
-        self.expand(stream)
+        self.select(stream)
         self.attention(stream, sm_scale)
         return self.out

@@ -24,7 +24,8 @@ QSA_DEV_BAD_REQUEST, QSA_DEV_TIMEOUT = 16, 32
 
 ENTRY_POINTS = (
     "qsa_index_scores", "qsa_topk_groups_workspace_size", "qsa_topk_groups",
-    "qsa_expand_select", "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
+    "qsa_expand_select", "qsa_topk_expand", "qsa_sparse_attn_decode_workspace_size",
+    "qsa_sparse_attn_decode",
     "qsa_sparse_attn_prefill", "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
 )
 
@@ -53,13 +54,14 @@ def lib() -> ctypes.CDLL:
     L.qsa_topk_groups_workspace_size.restype = U
     L.qsa_topk_groups.argtypes = [P, I, P, I, I, P, P, P, U, P, P]
     L.qsa_expand_select.argtypes = [P, P, I, P, P, I, P, P, I, P, P]
+    L.qsa_topk_expand.argtypes = [P, I, P, I, I, P, P, P, P, I, P, P]
     L.qsa_sparse_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
     L.qsa_sparse_attn_decode_workspace_size.restype = U
     L.qsa_sparse_attn_decode.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
                                          F, P, I, P, P, U, P, P]
     L.qsa_sparse_attn_prefill.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
                                           F, P, I, P, P, P]
-    for name in ("qsa_index_scores", "qsa_topk_groups", "qsa_expand_select",
+    for name in ("qsa_index_scores", "qsa_topk_groups", "qsa_expand_select", "qsa_topk_expand",
                  "qsa_sparse_attn_decode", "qsa_sparse_attn_prefill"):
         getattr(L, name).restype = I
     L.qsa_last_error_string.restype = ctypes.c_char_p
@@ -136,6 +138,15 @@ def qsa_expand_select(sel, n_sel, q_pos, tok, n_tok, capture_pos=None, dev_statu
         _ptr(sel), _ptr(n_sel), K, _ptr(q_pos), _ptr(capture_pos), T, _ptr(tok), _ptr(n_tok),
         tok.shape[1], _ptr(dev_status), _stream(stream)))
     return tok, n_tok
+
+
+def qsa_topk_expand(scores, q_pos, K, sel, n_sel, tok, n_tok, dev_status=None, stream=None):
+    """Top-K and expansion in one launch (rows without an MTP capture)."""
+    T, score_stride = scores.shape
+    _check(lib().qsa_topk_expand(
+        _ptr(scores), score_stride, _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel), _ptr(tok),
+        _ptr(n_tok), tok.shape[1], _ptr(dev_status), _stream(stream)))
+    return sel, n_sel, tok, n_tok
 
 
 def qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv_dtype=QSA_FP8_E4M3) -> int:

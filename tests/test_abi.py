@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 2
+    assert L.qsa_abi_version() == 3
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -89,6 +89,17 @@ def test_expand_validation(L):
     assert "4*K + 4" in _err(L)
     assert L.qsa_expand_select(NULL, NULL, 8, NULL, NULL, 1, NULL, NULL, 36, NULL, NULL) == 1
     assert L.qsa_expand_select(NULL, NULL, 8, NULL, NULL, 0, NULL, NULL, 36, NULL, NULL) == 0
+
+
+def test_topk_expand_validation(L):
+    # (scores, stride, q_pos, T, K, sel, n_sel, tok, n_tok, W, status, stream)
+    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 8, NULL, NULL, NULL, NULL, 35, NULL, NULL) == 1
+    assert "4*K + 4" in _err(L)
+    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 0, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
+    assert L.qsa_topk_expand(NULL, 10 ** 7, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 2
+    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
+    assert "null" in _err(L)
+    assert L.qsa_topk_expand(NULL, 16, NULL, 0, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 0
 
 
 def _attn(L, fn, T=1, Hq=16, Hkv=2, D=256, kv_dt=1, q_dt=1, out_dt=1, W=36, ks=1.0, vs=1.0,

@@ -173,6 +173,46 @@ def oracle_scores(n, rows, stride):
                             n["q_pos"][rows], n["q_req"][rows], stride)
 
 
+@pytest.mark.parametrize("case", ["tiny", "b1_16k", "dense_fallback", "prefill_rows", "odd_width"])
+def test_topk_expand_matches_separate_calls(case):
+    """qsa_topk_expand gives exactly the outputs of qsa_topk_groups followed
+    by qsa_expand_select, bit for bit, including the dense fallback (c <= K),
+    one-CTA rows (many queries) and a width that is not a multiple of 4."""
+    from indexer_top_sparse_c4_b200 import qsa
+    if case == "tiny":
+        w = wl.tiny(device="cuda")
+    elif case == "b1_16k":
+        w = wl.b1_16k(device="cuda")
+    elif case == "dense_fallback":   # 4,095 candidates, budget 8,192 groups
+        w = wl.b1_16k(device="cuda", K=8192)
+    else:
+        T, ctx = 300, 16384
+        pos = np.sort(np.random.default_rng(3).integers(4, ctx, T)).astype(np.int32)
+        w = wl.make("rows", B=1, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="bf16",
+                    q_dtype="bf16", seed=4, device="cuda", q_pos=pos, q_req=np.zeros(T, np.int32))
+    step = QSAStep(w)
+    step.index_scores()
+    W = w.W + (1 if case == "odd_width" else 0)
+    T, K = w.T, w.K
+    outs = []
+    for fused in (False, True):
+        sel = torch.full((T, K), 7, dtype=torch.int32, device="cuda")
+        n_sel = torch.full((T,), 7, dtype=torch.int32, device="cuda")
+        tok = torch.full((T, W), 7, dtype=torch.int32, device="cuda")
+        n_tok = torch.full((T,), 7, dtype=torch.int32, device="cuda")
+        status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        if fused:
+            qsa.qsa_topk_expand(step.scores, w.q_pos, K, sel, n_sel, tok, n_tok, dev_status=status)
+        else:
+            qsa.qsa_topk_groups(step.scores, w.q_pos, K, sel, n_sel, dev_status=status)
+            qsa.qsa_expand_select(sel, n_sel, w.q_pos, tok, n_tok, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        outs.append((sel, n_sel, tok, n_tok))
+    for x, y in zip(*outs):
+        assert torch.equal(x, y)
+
+
 def test_mtp_draft_reuse(oracle):
     w = wl.mtp(device="cuda")
     step = QSAStep(w)
