@@ -30,10 +30,12 @@
 // run's rows.  Scores of groups g >= c(p_t) inside a written tile are -inf.
 #include <cuda.h>
 
-#include "qsa_internal.cuh"
+#include "mbarrier.cuh"
 
 namespace qsa {
 namespace {
+
+using namespace mbar;
 
 constexpr int kQ = 128;                    // queries per M tile (TMEM lanes)
 constexpr int kH = 4;                      // indexer heads
@@ -51,7 +53,6 @@ constexpr int kBBytes = kKB * kBBlock;
 constexpr int kOutBytes = 32 * 32 * 4;     // a warp's 32 x 32 FP32 score block
 constexpr uint32_t kAccCols = kH * kN;     // 256 columns per accumulator set
 constexpr uint32_t kTmemCols = 2 * kAccCols;
-constexpr unsigned long long kWaitLimitNs = 200ull * 1000 * 1000;  // 200 ms per wait
 
 struct TcSmem {
   alignas(1024) unsigned char a[kABytes];
@@ -64,56 +65,6 @@ struct TcSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
-
-__device__ __forceinline__ uint32_t saddr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(saddr(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ unsigned long long gtimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait for the phase with the given parity; false (and the abort flag
-// set, QSA_DEV_TIMEOUT raised) when it does not come.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
-  const unsigned long long t0 = gtimer();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(b, parity)) return true;
-    if (*abort_flag) return false;
-    if ((i & 255u) == 255u && gtimer() - t0 > kWaitLimitNs) break;
-  }
-  *abort_flag = 1;
-  flag(status, QSA_DEV_TIMEOUT);
-  return false;
-}
-// After an abort: wait, with its own bound and whatever the abort flag says,
-// for a phase this thread armed, so that no copy or MMA still writes shared
-// memory or TMEM when the CTA leaves.
-__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
-  const unsigned long long t0 = gtimer();
-  for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(b, parity)) return;
-    if ((i & 255u) == 255u && gtimer() - t0 > kWaitLimitNs) return;
-  }
-}
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
@@ -282,9 +233,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hi = min(sh.nt_hi, run.ntiles);
         if (run.bad || sh.nt_lo >= hi) continue;
         if (!a_loaded) {
-          bool ok = true;
+          // the whole warp waits; one lane issues
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.a_empty, a_empty_par, abort_flag, a.status));
           if (lane == 0) {
-            ok = mbar_wait(&sm.a_empty, a_empty_par, abort_flag, a.status);
             if (ok) {
               mbar_arrive_tx(&sm.a_full, kABytes);
               for (int h = 0; h < kH; ++h)
@@ -292,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   tma_load_2d(sm.a + (h * kKB + kb) * kABlock, &tmap_q, &sm.a_full, h * kDI + kb * 64, t0);
             }
           }
-          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          if (!ok) break;
           a_armed = true;
           a_empty_par ^= 1;
           a_loaded = true;
@@ -307,12 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             page = lp < a.pt_stride ? __ldg(pt + lp) : -1;
             if (page < 0 || page >= a.num_pages) page = a.num_pages;
           }
-          bool ok = true;
-          if (lane == 0) {
-            ok = mbar_wait(&sm.b_empty[stage], bphase ^ 1, abort_flag, a.status);
-            if (ok) mbar_arrive_tx(&sm.b_full[stage], kBBytes);
-          }
-          if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+          const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.b_empty[stage], bphase ^ 1, abort_flag, a.status));
+          if (!ok) break;
+          if (lane == 0) mbar_arrive_tx(&sm.b_full[stage], kBBytes);
+          __syncwarp();
           if (lane < kNPages) {
             for (int kb = 0; kb < kKB; ++kb)
               tma_load_2d(sm.b[stage] + kb * kBBlock + lane * kPageGroups * 128, &tmap_k, &sm.b_full[stage],
@@ -346,16 +295,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hi = min(sh.nt_hi, run.ntiles);
         if (run.bad || sh.nt_lo >= hi) continue;
         if (!a_ready) {
-          if (lane == 0) ok = mbar_wait(&sm.a_full, aphase, abort_flag, a.status);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.a_full, aphase, abort_flag, a.status));
           if (!ok) break;
           aphase ^= 1;
           a_ready = true;
         }
         for (int nt = sh.nt_lo; nt < hi; ++nt) {
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_empty[abuf], accphase ^ 1, abort_flag, a.status) &&
+                                           mbar_wait(&sm.b_full[stage], bphase, abort_flag, a.status));
           if (lane == 0) {
-            ok = mbar_wait(&sm.acc_empty[abuf], accphase ^ 1, abort_flag, a.status) &&
-                 mbar_wait(&sm.b_full[stage], bphase, abort_flag, a.status);
             if (ok) {
               asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
               const uint32_t bbase = saddr(sm.b[stage]);
@@ -450,8 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const unsigned bad2 = __ballot_sync(0xffffffffu, pg < 0 || pg >= a.num_pages) & 3u;
           // when every row's candidates reach past these columns, no mask is needed
           const bool unmasked = __all_sync(0xffffffffu, !live || g0 + 32 <= c);
-          if (lane == 0) ok = mbar_wait(&sm.acc_full[abuf], accphase, abort_flag, a.status);
-          ok = __shfl_sync(0xffffffffu, ok, 0);
+          ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[abuf], accphase, abort_flag, a.status));
           if (!ok) break;
           asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
           // the previous TMA store must have read the staging block
