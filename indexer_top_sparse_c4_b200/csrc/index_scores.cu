@@ -46,6 +46,54 @@ __device__ __forceinline__ void warp_reduce_scatter(float* v, int lane) {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// L2 policies: the key stream (twice the L2 at B8 x 262,144 tokens) is read
+// once and marked evict-first, so it does not push out what the next stages
+// read right after it (the score rows, the page tables, the token lists); the
+// page-table entries are marked evict-last.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ int ldg_policy(const int32_t* p, uint64_t pol) {
+  int v;
+  asm volatile("ld.global.nc.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(v) : "l"(p), "l"(pol));
+  return v;
+}
+// VEC consecutive keys (element index i), widened to float, loaded with an L2 policy.
+template <typename KT, int VEC>
+__device__ __forceinline__ void ld_keys(const KT* base, size_t i, float* out, uint64_t pol) {
+  const void* p = base + i;
+  constexpr int B = VEC * (int)sizeof(KT);
+  uint32_t w[4];
+  if constexpr (B == 16) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.b32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "l"(p), "l"(pol));
+  } else if constexpr (B == 8) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v2.b32 {%0,%1}, [%2], %3;"
+                 : "=r"(w[0]), "=r"(w[1]) : "l"(p), "l"(pol));
+  } else if constexpr (B == 4) {
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b32 %0, [%1], %2;" : "=r"(w[0]) : "l"(p), "l"(pol));
+  } else {
+    unsigned short h;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(h) : "l"(p), "l"(pol));
+    w[0] = h;
+  }
+  if constexpr (sizeof(KT) == 4) {
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) out[e] = __uint_as_float(w[e]);
+  } else {  // BF16 pairs: the high half of an FP32 pattern
+#pragma unroll
+    for (int e = 0; e < VEC; ++e)
+      out[e] = __uint_as_float((e & 1) ? (w[e / 2] & 0xffff0000u) : (w[e / 2] << 16));
+  }
+}
+
 template <int H_I, int D_I, typename QT, typename KT>
 __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int warps_per_row) {
   constexpr int VEC = D_I / 32;          // dims per lane
@@ -78,12 +126,13 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
   for (int j = 0; j < R; ++j) w[j] = __ldg(a.w_idx + (size_t)t * H_I + (lane & 1) * R + j);
 
   const KT* kbase = reinterpret_cast<const KT*>(a.k_idx_pages);
+  const uint64_t pol_stream = l2_policy_evict_first(), pol_keep = l2_policy_evict_last();
   const int32_t* pt = a.page_table + (size_t)(bad_req ? 0 : r) * a.pt_stride;
   float* srow = a.scores + (size_t)t * a.score_stride;
 
   for (int lp = wid; lp < npages; lp += warps_per_row) {
     const int g = lp * kPageGroups + (lane >> 1);
-    const int page = (!bad_req && lp < a.pt_stride) ? __ldg(pt + lp) : -1;
+    const int page = (!bad_req && lp < a.pt_stride) ? ldg_policy(pt + lp, pol_keep) : -1;
     if (page < 0 || page >= a.num_pages) {  // warp-uniform
       if (lane == 0) flag(a.status, bad_req ? QSA_DEV_BAD_REQUEST : QSA_DEV_BAD_PAGE);
       if ((lane & 1) == 0 && g < c) srow[g] = -INFINITY;
@@ -92,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
     const KT* kp = kbase + (size_t)page * kPageGroups * D_I + lane * VEC;
     float k[kPageGroups][VEC];
 #pragma unroll
-    for (int gi = 0; gi < kPageGroups; ++gi) VecLoad<KT, VEC>::get(kp, (size_t)gi * D_I, k[gi]);
+    for (int gi = 0; gi < kPageGroups; ++gi) ld_keys<KT, VEC>(kp, (size_t)gi * D_I, k[gi], pol_stream);
     float acc[V];
 #pragma unroll
     for (int gi = 0; gi < kPageGroups; ++gi) {
