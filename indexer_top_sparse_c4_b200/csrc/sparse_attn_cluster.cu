@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
 
   // ---- merge the warps.  Per head (one thread each): the max over the warps
   // and every warp's rescale factor; then thread -> (head, 4 consecutive dims)
-  __shared__ float fac[NW][8];   // warp w's factor for head h (0: nothing to add)
+  __shared__ float fac[NW][8];   // warp w's factor for head h
   __shared__ float hml[8][2];    // the CTA's (max, sum) per head
   if (tid < 8) {
     const int h = tid;
@@ -380,9 +380,25 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
     hml[h][0] = M;
     hml[h][1] = L;
   }
+  // The cluster's outputs are split among its CTAs: CTA r finishes items
+  // [r * PER, (r + 1) * PER).  Every CTA pushes its share of item i (and its
+  // per-head max and sum) into the owner's receive slots before ONE cluster
+  // barrier; after it each CTA reads only its own shared memory.
+  constexpr int ITEMS8 = 8 * (D / 4);
+  constexpr int PER = (ITEMS8 + CL - 1) / CL;
+  __shared__ float4 recv_o[CL][PER];
+  __shared__ float recv_ml[CL][8][2];
   __syncthreads();
   const size_t th0 = (size_t)t * a.Hq + h0;
   const int items = G * (D / 4);
+  if constexpr (CL > 1) {
+    if (tid < 8 * CL) {
+      const int q = tid / 8, h = tid % 8;
+      float* dst = cl.map_shared_rank(&recv_ml[0][0][0], q);
+      dst[(rank * 8 + h) * 2] = hml[h][0];
+      dst[(rank * 8 + h) * 2 + 1] = hml[h][1];
+    }
+  }
   for (int idx = tid; idx < items; idx += NT) {
     const int h = idx / (D / 4), d = 4 * (idx % (D / 4));
     // every slot is written (zeros for warps without tiles): all loads go out at once
@@ -395,54 +411,47 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
       const float f = fac[w][h];
       O.x = fmaf(v[w].x, f, O.x); O.y = fmaf(v[w].y, f, O.y); O.z = fmaf(v[w].z, f, O.z); O.w = fmaf(v[w].w, f, O.w);
     }
-    if constexpr (CL == 1) write_out<OT, D>(a, th0 + h, d, O, hml[h][0], hml[h][1], vmul);
-    else st_o4<SH>(wo_dyn + h * OS, d, O);  // read above only by this thread
+    if constexpr (CL == 1) {
+      write_out<OT, D>(a, th0 + h, d, O, hml[h][0], hml[h][1], vmul);
+    } else {
+      const int owner = idx / PER;
+      *cl.map_shared_rank(&recv_o[rank][idx - owner * PER], owner) = O;
+    }
   }
   if constexpr (CL > 1) {
-    // ---- merge the cluster's CTAs: per head the cluster max and each CTA's
-    // factor (remote reads by 8 threads), then CTA `rank` finishes 1/CL of the outputs
+    cl.sync();  // every push has landed; from here every access is local
     __shared__ float cfac[CL][8];
     __shared__ float cml[8][2];
-    cl.sync();
     if (tid < 8) {
       const int h = tid;
-      float mq[CL], lq[CL];
       float M = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < CL; ++q) {
-        const float* r = cl.map_shared_rank(&hml[0][0], q);
-        mq[q] = r[h * 2];
-        lq[q] = r[h * 2 + 1];
-        M = fmaxf(M, mq[q]);
-      }
+      for (int q = 0; q < CL; ++q) M = fmaxf(M, recv_ml[q][h][0]);
       float L = 0.f;
 #pragma unroll
       for (int q = 0; q < CL; ++q) {
-        const float f = mq[q] == -INFINITY ? 0.f : exp2f(mq[q] - M);
+        const float mq = recv_ml[q][h][0];
+        const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
         cfac[q][h] = f;
-        L = fmaf(lq[q], f, L);
+        L = fmaf(recv_ml[q][h][1], f, L);
       }
       cml[h][0] = M;
       cml[h][1] = L;
     }
     __syncthreads();
-    const int per = (items + CL - 1) / CL;
-    const int lo = rank * per;
-    const int hi = lo + per < items ? lo + per : items;
+    const int lo = rank * PER;
+    const int hi = lo + PER < items ? lo + PER : items;
     for (int idx = lo + tid; idx < hi; idx += NT) {
       const int h = idx / (D / 4), d = 4 * (idx % (D / 4));
-      float4 v[CL];
-#pragma unroll
-      for (int q = 0; q < CL; ++q) v[q] = ld_o4<SH>(cl.map_shared_rank(wo_dyn + h * OS, q), d);
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < CL; ++q) {
         const float f = cfac[q][h];
-        O.x = fmaf(v[q].x, f, O.x); O.y = fmaf(v[q].y, f, O.y); O.z = fmaf(v[q].z, f, O.z); O.w = fmaf(v[q].w, f, O.w);
+        const float4 v = recv_o[q][idx - lo];
+        O.x = fmaf(v.x, f, O.x); O.y = fmaf(v.y, f, O.y); O.z = fmaf(v.z, f, O.z); O.w = fmaf(v.w, f, O.w);
       }
       write_out<OT, D>(a, th0 + h, d, O, cml[h][0], cml[h][1], vmul);
     }
-    cl.sync();  // peers may read this CTA's shared memory until here
   }
 }
 
