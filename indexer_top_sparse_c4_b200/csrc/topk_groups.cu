@@ -36,12 +36,16 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
 constexpr int kMaxCL = 8;
 
+constexpr int kCandCap = 2048;  // candidates gathered after two passes (else four cluster passes)
+
 struct TopkSmem {
   uint32_t hw[kWarps][kBins];            // per-warp histogram of the current digit
   uint32_t hall[4][kMaxCL][kBins];       // per pass: slot q = CTA q's histogram
+  uint2 cand[kCandCap];                  // (key, id) of every candidate of the cluster
   int wsum[kWarps][kMaxCL];              // block reduction of the per-CTA counts above tau
+  int ccnt[2 * kMaxCL];                  // per CTA: candidates above tau, equal to tau
   int wa[kWarps];                        // per-warp scan totals
-  int bin[4], above;
+  int bin[4], above[4];
 };
 
 // float -> uint32 whose unsigned order equals the float order; -0 maps like +0.
@@ -78,6 +82,27 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
     total += x;
   }
   return before + incl - v;
+}
+
+// Threads 0..255 (warps 0..7) hold the counts h of the bins 255 - tid, i.e.
+// from the top: the thread whose bin holds the need-th largest key writes the
+// bin and the count of keys in all higher bins.
+__device__ __forceinline__ void find_bin(int h, int need, int my_bin, int* bin_out, int* above_out, int* wa) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = h;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += u;
+  }
+  if (lane == 31) wa[warp] = incl;
+  asm volatile("bar.sync 1, %0;" ::"r"(kBins));  // the 8 warps that scan
+  int above = incl - h;
+  for (int w = 0; w < warp; ++w) above += wa[w];
+  if (above < need && above + h >= need) {
+    *bin_out = my_bin;
+    *above_out = above;
+  }
 }
 
 template <int CL, int KPT>
@@ -137,9 +162,14 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
   }
   pdl_launch_dependents();
 
-  // ---- radix select: 4 passes of 8 bits locate tau
+  // ---- radix select: passes of 8 bits from the top locate tau.  After two
+  // cluster passes the keys that still match (the candidates) are usually a
+  // few dozen; then every CTA receives all of them and finishes the last two
+  // digits on its own, without further cluster barriers.
   uint32_t prefix = 0;
   int need = n;  // how many keys matching `prefix` are still to be taken
+  int npass = 4;  // cluster passes whose tables count the keys above tau
+  int ncand = 0;
 #pragma unroll
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
@@ -166,44 +196,88 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
       }
     }
     csync<CL>();  // every CTA's counts are in every CTA's table
-    // the bin holding the need-th largest: thread i looks at bin 255 - i, so
-    // an exclusive scan over threads counts the keys in all higher bins
     if (tid < kBins) {
       int h = 0;
 #pragma unroll
       for (int q = 0; q < CL; ++q) h += (int)sm.hall[pass][q][kBins - 1 - tid];
-      int incl = h;
-#pragma unroll
-      for (int d = 1; d < 32; d <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, d);
-        if (lane >= d) incl += u;
-      }
-      if (lane == 31) sm.wa[warp] = incl;
-      asm volatile("bar.sync 1, %0;" ::"r"(kBins));  // the 8 warps that scan
-      int above = incl - h;
-      for (int w = 0; w < warp; ++w) above += sm.wa[w];
-      if (above < need && above + h >= need) {
-        sm.bin[pass] = kBins - 1 - tid;
-        sm.above = above;
-      }
+      find_bin(h, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
     }
     __syncthreads();
     prefix |= (uint32_t)sm.bin[pass] << shift;
-    need -= sm.above;
-    __syncthreads();
+    need -= sm.above[pass];
+    if (CL > 1 && pass == 1) {  // (a one-CTA row keeps its four passes)
+      int total = 0;
+#pragma unroll
+      for (int q = 0; q < CL; ++q) total += (int)sm.hall[1][q][sm.bin[1]];
+      if (total <= kCandCap) {  // the same decision in every CTA
+        npass = 2;
+        ncand = total;
+        break;
+      }
+    }
+  }
+
+  if constexpr (CL > 1) if (npass == 2) {
+    // ---- candidates: every CTA writes its keys matching the 16-bit prefix,
+    // with their ids, into every CTA's list (CTA q's block starts after the
+    // candidates of CTAs 0 .. q-1, whose counts pass 1's table holds)
+    int mine = 0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) mine += (keys[j] >> 16) == (prefix >> 16);
+    int cta_total;
+    int pos = block_exclusive_scan(mine, sm.wa, cta_total);
+    for (int q = 0; q < rank; ++q) pos += (int)sm.hall[1][q][sm.bin[1]];
+    if (mine) {
+      cg::cluster_group cl = cg::this_cluster();
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) {
+        if ((keys[j] >> 16) == (prefix >> 16)) {
+          const uint2 e = make_uint2(keys[j], (uint32_t)(first + j));
+          for (int q = 0; q < CL; ++q) *cl.map_shared_rank(&sm.cand[pos], q) = e;
+          ++pos;
+        }
+      }
+    }
+    if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
+    csync<CL>();  // the lists are complete; from here every access is local
+    // ---- the last two digits, over the candidates only
+#pragma unroll
+    for (int pass = 2; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      if (tid < kBins) sm.hw[0][tid] = 0u;
+      __syncthreads();
+      for (int i = tid; i < ncand; i += kThreads) {
+        const uint32_t k = sm.cand[i].x;
+        if ((k >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&sm.hw[0][(k >> shift) & (kBins - 1)], 1u);
+      }
+      __syncthreads();
+      if (tid < kBins)
+        find_bin((int)sm.hw[0][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+      __syncthreads();
+      prefix |= (uint32_t)sm.bin[pass] << shift;
+      need -= sm.above[pass];
+    }
+    // per-CTA counts of candidates above and equal to tau (the CTA owning an id)
+    for (int i = tid; i < ncand; i += kThreads) {
+      const uint2 e = sm.cand[i];
+      const int q = (int)(e.y / (uint32_t)(kThreads * KPT));
+      if (e.x > prefix) atomicAdd(&sm.ccnt[q], 1);
+      else if (e.x == prefix) atomicAdd(&sm.ccnt[kMaxCL + q], 1);
+    }
   }
   const uint32_t tau = prefix;
 
   // ---- keys above tau in each CTA: a key is above tau when, in the first
   // pass where its digit differs from tau's, its digit is the larger one, and
-  // that pass's table counted it under that digit in its CTA's slot
+  // that pass's table counted it under that digit in its CTA's slot (on the
+  // candidate path the last two passes are counted from the candidate list)
   if (tid < kBins) {
     int x[kMaxCL];
 #pragma unroll
     for (int q = 0; q < CL; ++q) x[q] = 0;
 #pragma unroll
     for (int pass = 0; pass < 4; ++pass) {
-      if (tid > sm.bin[pass]) {
+      if (pass < npass && tid > sm.bin[pass]) {
 #pragma unroll
         for (int q = 0; q < CL; ++q) x[q] += (int)sm.hall[pass][q][tid];
       }
@@ -224,14 +298,14 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
     eq += keys[j] == tau;
   }
   int both;  // one scan of gt (low 16 bits) and eq (high): per-CTA counts stay below 2^16
-  const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum visible
+  const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum, ccnt visible
   const int gt_before = before & 0xffff, eq_before = before >> 16;
   int off = 0, eq_prev = 0;
   for (int q = 0; q < rank; ++q) {
-    int gt_q = 0;
+    int gt_q = npass == 2 ? sm.ccnt[q] : 0;
 #pragma unroll
     for (int w = 0; w < kBins / 32; ++w) gt_q += sm.wsum[w][q];
-    const int eq_q = (int)sm.hall[3][q][sm.bin[3]];
+    const int eq_q = npass == 2 ? sm.ccnt[kMaxCL + q] : (int)sm.hall[3][q][sm.bin[3]];
     const int rem = need - eq_prev;
     off += gt_q + (rem <= 0 ? 0 : (rem < eq_q ? rem : eq_q));
     eq_prev += eq_q;
