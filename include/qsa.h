@@ -90,7 +90,8 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
  * For every query token t and complete group g < c = q_pos[t]/4 (capped at
  * score_stride):  scores[t*score_stride + g] = sum_h w_idx[t,h] *
  * ReLU(q_idx[t,h,:] . khat[g,:]), computed in FP32.  khat[g] is row g%16 of
- * page page_table[q_req[t]][g/16].  Entries g >= c are not written.  A group
+ * page page_table[q_req[t]][g/16].  Entries g >= c are either left as they
+ * are or set to -inf (the tensor-core pass writes whole tiles).  A group
  * whose page id is out of range scores -inf and sets QSA_DEV_BAD_PAGE.
  * Supported: H_I in {2, 4}, D_I in {32, 64, 128}, q_dt and k_dt F32 or BF16.
  * The score formula is the one this library fixes for the learned compressed
@@ -154,12 +155,12 @@ QSA_API qsa_status_t qsa_topk_expand(const float* scores, int score_stride, cons
  * sm_scale <= 0.  lse may be NULL.
  * Supported: D in {64, 128, 256}, Hq/Hkv <= 16, q_dt F32 or BF16, kv_dt F32,
  * BF16 or FP8_E4M3, out_dt F32 or BF16.
- * _decode splits every row's tokens across CTAs (split-K): the CTAs of a
- * thread-block cluster merge their partials on chip; when a call needs more
- * than one cluster per (query, KV head) the clusters' partials go through
- * qsa_sparse_attn_decode_workspace_size(..., kv_dt) bytes of workspace (0 when
- * none is needed).  _prefill gives each (query, KV head) its own CTA and needs
- * no workspace. */
+ * _decode splits every row's tokens across the CTAs of one thread-block
+ * cluster per (query, KV head), which merge their partials on chip; only
+ * rows too long for one cluster are split over several, whose partials go
+ * through qsa_sparse_attn_decode_workspace_size(..., kv_dt) bytes of
+ * workspace (0 when none is needed).  _prefill gives each (query, KV head)
+ * its own warp and needs no workspace. */
 QSA_API size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W,
                                                      qsa_dtype_t kv_dt);
 QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
