@@ -103,7 +103,8 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
   const int lane = threadIdx.x & 31;
   const int wid = blockIdx.x * kWarps + (threadIdx.x >> 5);
   pdl_wait();
-  pdl_launch_dependents();  // the next kernel's CTAs may take SMs this grid's last wave leaves free
+  // (no early trigger: the dependents launch when this grid completes; launched
+  // earlier, their CTAs took SMs from this grid's later waves)
   const int p = a.q_pos[t];
   int c = p >= 0 ? p / kGroupTokens : 0;
   if (c > a.score_stride) {

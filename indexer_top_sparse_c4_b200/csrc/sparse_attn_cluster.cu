@@ -207,7 +207,6 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
         for (int u = 0; u < 4; ++u) vr[i][u][j] = oV[u] >= 0 ? ldg16(vbase + oV[u] + cb) : z;
       }
     }
-    if (k0 == 0) pdl_launch_dependents();
 
     // ---- S^T = K . Q^T per tile: s[i][0], s[i][1] token g, heads 2tq, 2tq+1;
     // s[i][2], s[i][3] token g+8
@@ -349,7 +348,6 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
     first = false;
   }
   if (first) {  // a warp without tiles: its slot holds zeros, so merges need no branch
-    pdl_launch_dependents();
     for (int i = lane; i < 8 * OS / 4; i += 32) reinterpret_cast<float4*>(wow)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   if (g == 0) {

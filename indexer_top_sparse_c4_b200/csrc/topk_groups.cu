@@ -160,7 +160,8 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
       for (int e = 0; e < 4; ++e) keys[j + e] = first + j + e < c ? order_key(__ldg(row + first + j + e)) : 0u;
     }
   }
-  pdl_launch_dependents();
+  // (dependents launch when this grid completes: launched earlier, their CTAs
+  // compete for the SMs this kernel still needs)
 
   // ---- radix select: passes of 8 bits from the top locate tau.  After two
   // cluster passes the keys that still match (the candidates) are usually a
