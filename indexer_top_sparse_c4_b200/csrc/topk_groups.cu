@@ -37,6 +37,7 @@ constexpr int kBins = 256;
 constexpr int kMaxCL = 8;
 
 constexpr int kCandCap = 2048;  // candidates gathered after two passes (else four cluster passes)
+constexpr int kRankCap = 512;   // up to this many candidates are ranked directly
 
 struct TopkSmem {
   uint32_t hw[kWarps][kBins];            // per-warp histogram of the current digit
@@ -46,6 +47,7 @@ struct TopkSmem {
   int ccnt[2 * kMaxCL];                  // per CTA: candidates above tau, equal to tau
   int wa[kWarps];                        // per-warp scan totals
   int bin[4], above[4];
+  uint32_t tau;
 };
 
 // float -> uint32 whose unsigned order equals the float order; -0 maps like +0.
@@ -241,22 +243,43 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
     }
     if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
     csync<CL>();  // the lists are complete; from here every access is local
-    // ---- the last two digits, over the candidates only
-#pragma unroll
-    for (int pass = 2; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      if (tid < kBins) sm.hw[0][tid] = 0u;
-      __syncthreads();
-      for (int i = tid; i < ncand; i += kThreads) {
-        const uint32_t k = sm.cand[i].x;
-        if ((k >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&sm.hw[0][(k >> shift) & (kBins - 1)], 1u);
+    if (ncand <= kRankCap) {
+      // ---- few candidates: the rank of each under (key desc, id asc) is a
+      // direct count; the candidate of rank need-1 is tau
+      if (tid < ncand) {
+        const uint2 me = sm.cand[tid];
+        int r = 0, r_key = 0;  // rank, and candidates with a larger key
+        for (int i = 0; i < ncand; ++i) {
+          const uint2 o = sm.cand[i];
+          r += o.x > me.x || (o.x == me.x && o.y < me.y);
+          r_key += o.x > me.x;
+        }
+        if (r == need - 1) {
+          sm.tau = me.x;
+          sm.above[2] = r_key;  // candidates above tau
+        }
       }
       __syncthreads();
-      if (tid < kBins)
-        find_bin((int)sm.hw[0][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
-      __syncthreads();
-      prefix |= (uint32_t)sm.bin[pass] << shift;
-      need -= sm.above[pass];
+      prefix = sm.tau;
+      need -= sm.above[2];
+    } else {
+      // ---- the last two digits, over the candidates only
+#pragma unroll
+      for (int pass = 2; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        if (tid < kBins) sm.hw[0][tid] = 0u;
+        __syncthreads();
+        for (int i = tid; i < ncand; i += kThreads) {
+          const uint32_t k = sm.cand[i].x;
+          if ((k >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&sm.hw[0][(k >> shift) & (kBins - 1)], 1u);
+        }
+        __syncthreads();
+        if (tid < kBins)
+          find_bin((int)sm.hw[0][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+        __syncthreads();
+        prefix |= (uint32_t)sm.bin[pass] << shift;
+        need -= sm.above[pass];
+      }
     }
     // per-CTA counts of candidates above and equal to tau (the CTA owning an id)
     for (int i = tid; i < ncand; i += kThreads) {
@@ -301,21 +324,39 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
   int both;  // one scan of gt (low 16 bits) and eq (high): per-CTA counts stay below 2^16
   const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum, ccnt visible
   const int gt_before = before & 0xffff, eq_before = before >> 16;
+  // the CTAs before this one: lane q of every warp takes CTA q's counts, and a
+  // warp prefix over q gives the offsets (no serial loop, no extra barrier)
   int off = 0, eq_prev = 0;
-  for (int q = 0; q < rank; ++q) {
-    int gt_q = npass == 2 ? sm.ccnt[q] : 0;
+  if constexpr (CL > 1) {
+    int gt_q = 0, eq_q = 0;
+    if (lane < CL) {
+      gt_q = npass == 2 ? sm.ccnt[lane] : 0;
 #pragma unroll
-    for (int w = 0; w < kBins / 32; ++w) gt_q += sm.wsum[w][q];
-    const int eq_q = npass == 2 ? sm.ccnt[kMaxCL + q] : (int)sm.hall[3][q][sm.bin[3]];
-    const int rem = need - eq_prev;
-    off += gt_q + (rem <= 0 ? 0 : (rem < eq_q ? rem : eq_q));
-    eq_prev += eq_q;
+      for (int w = 0; w < kBins / 32; ++w) gt_q += sm.wsum[w][lane];
+      eq_q = npass == 2 ? sm.ccnt[kMaxCL + lane] : (int)sm.hall[3][lane][sm.bin[3]];
+    }
+    // exclusive prefix over lanes q < rank of the kept count: gt_q plus the
+    // tau-keys CTA q takes, which depends on the tau-keys before it
+    int eq_incl = eq_q;
+#pragma unroll
+    for (int d = 1; d < kMaxCL; d <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, eq_incl, d);
+      if (lane >= d) eq_incl += u;
+    }
+    const int eq_before_q = eq_incl - eq_q;
+    const int rem_q = need - eq_before_q;
+    int kept_q = lane < rank ? gt_q + (rem_q <= 0 ? 0 : (rem_q < eq_q ? rem_q : eq_q)) : 0;
+#pragma unroll
+    for (int d = 1; d < kMaxCL; d <<= 1) kept_q += __shfl_xor_sync(0xffffffffu, kept_q, d);
+    off = __shfl_sync(0xffffffffu, kept_q, 0);
+    eq_prev = __shfl_sync(0xffffffffu, eq_before_q, rank);
   }
   int rem = need - eq_prev;                     // tau-keys still to take at this CTA's start
   rem = rem < 0 ? 0 : rem;
   int pos = off + gt_before + (rem < eq_before ? rem : eq_before);
   int take = rem - eq_before;                   // tau-keys this thread may take
   take = take < 0 ? 0 : take;
+  if (gt > 0 || take > 0)  // (most threads keep nothing)
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
     const uint32_t k = keys[j];
