@@ -194,7 +194,7 @@ struct DecodePlan {
 };
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
-// decode == true: the split plan is used; otherwise (prefill) one CTA per
+// decode == true: the decode plan is used; otherwise (prefill) one warp per
 // (query, KV head) row streams all of its tokens.
 cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
                                bool decode);
@@ -206,17 +206,17 @@ bool attn_mma_supported(const AttnArgs& a);
 // row: no workspace, no combine.  Token slots one pass of the kernel covers
 // per warp step (larger rows take several steps).
 int attn_cluster_tokens_per_round(qsa_dtype_t kv_dt, int D, int cl);
+// Many rows: one warp per (query, KV head) row with all its query heads,
+// K/V streamed through a per-warp cp.async ring.
+cudaError_t launch_sparse_attn_prefill_rows(const AttnArgs& a, float qk_scale_log2, float vmul, cudaStream_t s);
 cudaError_t launch_sparse_attn_cluster(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                        cudaStream_t s);
-// Decode kernel on the same tensor-core tiles: one 16-token tile per warp,
-// attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on chip.
+// Decode kernel for rows too long for one cluster: one 16-token tile per
+// warp, attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on
+// chip, cluster groups merged by the combine kernel.
 int attn_tile_tokens();
-cudaError_t launch_sparse_attn_rowwarp(const AttnArgs& a, float qk_scale_log2, float vmul,
-                                       cudaStream_t stream);
 cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                     int s, void* ws, cudaStream_t stream);
-cudaError_t launch_sparse_attn_mma(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
-                                   int s, void* ws, cudaStream_t stream);
 
 // Sets the message qsa_last_error_string() returns on this thread.
 void set_last_error(const char* msg);

@@ -344,7 +344,7 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   sc.vmul = fp8 ? a.v_scale : 1.f;
   cudaError_t e;
   if (attn_mma_supported(a)) {
-    e = plan.stream    ? launch_sparse_attn_rowwarp(a, sc.qk, sc.vmul, s)
+    e = plan.stream    ? launch_sparse_attn_prefill_rows(a, sc.qk, sc.vmul, s)
         : plan.cluster ? launch_sparse_attn_cluster(a, sc.qk, sc.vmul, plan.cl, s)
                        : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
   } else {
