@@ -223,23 +223,29 @@ def time_steps(sets, steps, warmup, stream):
 def time_stages(sets, reps, stream):
     """Per-stage device times (us).  `alone`: a graph of `reps` launches of that
     stage only (for the indexer scan every launch streams its 256 MiB of keys
-    from HBM, so this is its true launch duration).  `in_step`: what the stage
+    from HBM, so this is its true launch duration).  The Top-K consumes the
+    prefix histogram the scan leaves, so it is timed after the scan: the graph
+    of (scan, Top-K) pairs minus the graph of scans.  `in_step`: what the stage
     adds to a step, i.e. the step graph minus the same graph without it."""
+    def timed(stages):
+        g = capture(sets, reps, stages)
+        g.replay()
+        ms = replay_ms(g)
+        del g
+        for st in sets:   # graphs without the Top-K leave the histogram counted up
+            if st.prefix_hist is not None:
+                st.prefix_hist.zero_()
+        return ms
+
     alone, in_step = {}, {}
     with torch.cuda.stream(stream):
-        full = capture(sets, reps)
-        full.replay()
-        t_full = replay_ms(full)
-        del full
+        t_full = timed(STAGES)
         for name in STAGES:
-            g = capture(sets, reps, (name,))
-            g.replay()
-            alone[name] = replay_ms(g) / reps * 1e3
-            del g
-            g = capture(sets, reps, tuple(x for x in STAGES if x != name))
-            g.replay()
-            in_step[name] = (t_full - replay_ms(g)) / reps * 1e3
-            del g
+            if name == "select" and sets[0].prefix_hist is not None:
+                alone[name] = (timed(("index_scores", "select")) - timed(("index_scores",))) / reps * 1e3
+            else:
+                alone[name] = timed((name,)) / reps * 1e3
+            in_step[name] = (t_full - timed(tuple(x for x in STAGES if x != name))) / reps * 1e3
     return alone, in_step
 
 

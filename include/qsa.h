@@ -86,6 +86,13 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
 #define QSA_DEV_TIMEOUT 32u   /* a bounded wait inside a kernel ran out (the
                                  kernel stopped early; its outputs are invalid) */
 
+/* Width of one row of the optional prefix histogram passed from stage 1 to
+ * stage 2 (prefix_hist below): one uint32 count per value of the top 12 bits
+ * of a score's order key.  The order key of a float is its bit pattern with
+ * the sign bit set when the sign is clear, and with every bit flipped when the
+ * sign is set (-0.0 counts as +0.0): unsigned key order is score order. */
+#define QSA_PREFIX_HIST_BINS 4096
+
 /* Stage 1 -- indexer scores.
  * For every query token t and complete group g < c = q_pos[t]/4 (capped at
  * score_stride):  scores[t*score_stride + g] = sum_h w_idx[t,h] *
@@ -95,13 +102,20 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
  * whose page id is out of range scores -inf and sets QSA_DEV_BAD_PAGE.
  * Supported: H_I in {2, 4}, D_I in {32, 64, 128}, q_dt and k_dt F32 or BF16.
  * The score formula is the one this library fixes for the learned compressed
- * indexer ("QSA in brief" names the indexer, not its formula). */
+ * indexer ("QSA in brief" names the indexer, not its formula).
+ * prefix_hist (optional; NULL = not used): [T, QSA_PREFIX_HIST_BINS] uint32,
+ * all zero on entry.  The streaming scan (the pass used unless T >= 256 with
+ * BF16 query and keys, H_I = 4, D_I = 128) adds to row t one count per score
+ * it writes, in the bin of the score's top 12 order-key bits.  The tensor-core
+ * pass leaves the buffer as it is.  Given to the Top-K call that reads these
+ * scores, the histogram replaces that call's first radix passes; the Top-K
+ * call zeroes it again. */
 QSA_API qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
                               const int32_t* page_table, int pt_rows, int pt_stride,
                               const int32_t* q_req, const int32_t* q_pos, int T, int H_I,
-                              int D_I, float* scores, int score_stride, uint32_t* dev_status,
-                              qsa_stream_t stream);
+                              int D_I, float* scores, int score_stride, uint32_t* prefix_hist,
+                              uint32_t* dev_status, qsa_stream_t stream);
 
 /* Stage 2 -- exact Top-K over compressed groups (TensorRT-LLM
  * "QSASparseAttentionConfig", enable_heuristic_topk: the exact radix Top-K).
@@ -110,11 +124,17 @@ QSA_API qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const
  * lower group id (-0.0 ranks equal to +0.0; scores must not be NaN).
  * sel [T, K] receives the kept group ids in ascending order followed by -1;
  * n_sel [T] receives n.  c <= K keeps every candidate (dense fallback).
- * workspace: qsa_topk_groups_workspace_size() bytes (may be 0 / NULL). */
+ * workspace: qsa_topk_groups_workspace_size() bytes (may be 0 / NULL).
+ * prefix_hist (optional; NULL = not used): the histogram qsa_index_scores
+ * built while writing these scores, unchanged since.  A row whose histogram
+ * total equals its candidate count c takes the bin of its n-th largest key
+ * from it instead of from radix passes over the scores; any other row runs
+ * the full passes.  The outputs are the same either way.  On return rows
+ * 0..T-1 of prefix_hist are zero, ready for the next qsa_index_scores. */
 QSA_API size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride);
-QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, const int32_t* q_pos,
-                             int T, int K, int32_t* sel, int32_t* n_sel, void* workspace,
-                             size_t workspace_bytes, uint32_t* dev_status,
+QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint32_t* prefix_hist,
+                             const int32_t* q_pos, int T, int K, int32_t* sel, int32_t* n_sel,
+                             void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                              qsa_stream_t stream);
 
 /* Stage 3 -- expansion of the kept groups to token ids ("QSA in brief": the
@@ -133,14 +153,16 @@ QSA_API qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel,
                                qsa_stream_t stream);
 
 /* Stages 2 and 3 in one launch, for rows without an MTP capture: exactly
- * qsa_topk_groups(scores, score_stride, q_pos, T, K, sel, n_sel) followed by
- * qsa_expand_select(sel, n_sel, K, q_pos, NULL, T, tok, n_tok, W), with the
- * same outputs, layouts and status bits.  The expansion is not defined by
- * the pages as a separate pass: joining it to the selection saves a launch
- * and a read of sel on the decode path.  W >= 4*K + 4. */
-QSA_API qsa_status_t qsa_topk_expand(const float* scores, int score_stride, const int32_t* q_pos, int T,
-                             int K, int32_t* sel, int32_t* n_sel, int32_t* tok, int32_t* n_tok,
-                             int W, uint32_t* dev_status, qsa_stream_t stream);
+ * qsa_topk_groups(scores, score_stride, prefix_hist, q_pos, T, K, sel, n_sel)
+ * followed by qsa_expand_select(sel, n_sel, K, q_pos, NULL, T, tok, n_tok, W),
+ * with the same outputs, layouts and status bits (prefix_hist as there).  The
+ * expansion is not defined by the pages as a separate pass: joining it to the
+ * selection saves a launch and a read of sel on the decode path.
+ * W >= 4*K + 4. */
+QSA_API qsa_status_t qsa_topk_expand(const float* scores, int score_stride, uint32_t* prefix_hist,
+                             const int32_t* q_pos, int T, int K, int32_t* sel, int32_t* n_sel,
+                             int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
+                             qsa_stream_t stream);
 
 /* Stage 4 -- GQA attention over the selected tokens ("QSA in brief": only the
  * selected entries are read; the Ascend article: rows with nothing to attend
@@ -212,7 +234,8 @@ QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */
 QSA_API const char* qsa_status_name(qsa_status_t s);
 /* ABI version: bumped on any change of the entry points (2: the decode
- * workspace query takes the KV dtype; 3: qsa_topk_expand). */
+ * workspace query takes the KV dtype; 3: qsa_topk_expand; 4: the prefix_hist
+ * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -13,6 +13,12 @@
 // reduce-scatter leaves lane l holding the finished dots of group l/2 for
 // H_I/2 heads; one more shuffle adds the head pair.  Shuffles per group:
 // ~H_I, against 5*H_I for a plain per-group warp reduction.
+//
+// Optionally the scan also counts its scores by the top 12 bits of their
+// order keys (the prefix histogram of the row): a shared-memory histogram per
+// CTA, added into the row's global one when the CTA ends.  The Top-K stage
+// then knows which 12-bit bin holds the n-th largest score without a pass of
+// its own over the row.
 #include "qsa_internal.cuh"
 
 namespace qsa {
@@ -95,24 +101,11 @@ __device__ __forceinline__ void ld_keys(const KT* base, size_t i, float* out, ui
 }
 
 template <int H_I, int D_I, typename QT, typename KT>
-__global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int warps_per_row) {
+__device__ __forceinline__ void scan_row(const IndexArgs& a, int t, int c, int npages, int wid, int lane,
+                                         int warps_per_row, uint32_t* hist_s) {
   constexpr int VEC = D_I / 32;          // dims per lane
   constexpr int V = kPageGroups * H_I;   // partial dots per lane per page
   constexpr int R = V / 32;              // finished dots per lane (= H_I / 2)
-  const int t = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  const int wid = blockIdx.x * kWarps + (threadIdx.x >> 5);
-  pdl_wait();
-  // (no early trigger: the dependents launch when this grid completes; launched
-  // earlier, their CTAs took SMs from this grid's later waves)
-  const int p = a.q_pos[t];
-  int c = p >= 0 ? p / kGroupTokens : 0;
-  if (c > a.score_stride) {
-    if (wid == 0 && lane == 0) flag(a.status, QSA_DEV_ROW_RANGE);
-    c = a.score_stride;
-  }
-  const int npages = (c + kPageGroups - 1) / kPageGroups;
-  if (wid >= npages) return;
   const int r = a.q_req ? a.q_req[t] : t;
   const bool bad_req = r < 0 || r >= a.pt_rows;  // every group of the row is skipped
 
@@ -136,7 +129,10 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
     const int page = (!bad_req && lp < a.pt_stride) ? ldg_policy(pt + lp, pol_keep) : -1;
     if (page < 0 || page >= a.num_pages) {  // warp-uniform
       if (lane == 0) flag(a.status, bad_req ? QSA_DEV_BAD_REQUEST : QSA_DEV_BAD_PAGE);
-      if ((lane & 1) == 0 && g < c) srow[g] = -INFINITY;
+      if ((lane & 1) == 0 && g < c) {
+        srow[g] = -INFINITY;
+        if (hist_s) atomicAdd(&hist_s[order_key(-INFINITY) >> kPrefixShift], 1u);
+      }
       continue;
     }
     const KT* kp = kbase + (size_t)page * kPageGroups * D_I + lane * VEC;
@@ -159,7 +155,46 @@ __global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int
 #pragma unroll
     for (int j = 0; j < R; ++j) s = fmaf(w[j], fmaxf(acc[j], 0.f), s);
     s += __shfl_xor_sync(0xffffffffu, s, 1);
-    if ((lane & 1) == 0 && g < c) srow[g] = s;
+    if ((lane & 1) == 0 && g < c) {
+      srow[g] = s;
+      if (hist_s) atomicAdd(&hist_s[order_key(s) >> kPrefixShift], 1u);
+    }
+  }
+}
+
+template <int H_I, int D_I, typename QT, typename KT>
+__global__ void __launch_bounds__(kThreads) index_scores_kernel(IndexArgs a, int warps_per_row) {
+  __shared__ __align__(16) uint32_t hist_s[kPrefixBins];
+  const int t = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int wid = blockIdx.x * kWarps + (threadIdx.x >> 5);
+  pdl_wait();
+  // (no early trigger: the dependents launch when this grid completes; launched
+  // earlier, their CTAs took SMs from this grid's later waves)
+  const int p = a.q_pos[t];
+  int c = p >= 0 ? p / kGroupTokens : 0;
+  if (c > a.score_stride) {
+    if (wid == 0 && lane == 0) flag(a.status, QSA_DEV_ROW_RANGE);
+    c = a.score_stride;
+  }
+  const int npages = (c + kPageGroups - 1) / kPageGroups;
+  if (blockIdx.x * kWarps >= npages) return;  // (CTA-uniform: before any barrier)
+  uint32_t* const hist_g = a.hist ? a.hist + (size_t)t * kPrefixBins : nullptr;
+  if (hist_g) {
+#pragma unroll
+    for (int i = 4 * threadIdx.x; i < kPrefixBins; i += 4 * kThreads)
+      *reinterpret_cast<uint4*>(&hist_s[i]) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+  }
+  if (wid < npages) scan_row<H_I, D_I, QT, KT>(a, t, c, npages, wid, lane, warps_per_row,
+                                               hist_g ? hist_s : nullptr);
+  if (hist_g) {  // the CTA's counts into the row's histogram (few bins are non-zero)
+    __syncthreads();
+#pragma unroll 4
+    for (int i = threadIdx.x; i < kPrefixBins; i += kThreads) {
+      const uint32_t v = hist_s[i];
+      if (v) atomicAdd(hist_g + i, v);
+    }
   }
 }
 

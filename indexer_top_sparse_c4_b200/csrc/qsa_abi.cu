@@ -82,14 +82,15 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 3; }
+int qsa_abi_version(void) { return 4; }
 
 qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
                               const int32_t* page_table, int pt_rows, int pt_stride,
                               const int32_t* q_req,
                               const int32_t* q_pos, int T, int H_I, int D_I, float* scores,
-                              int score_stride, uint32_t* dev_status, qsa_stream_t stream) {
+                              int score_stride, uint32_t* prefix_hist, uint32_t* dev_status,
+                              qsa_stream_t stream) {
   REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
   SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
   SUPPORT((H_I == 2 || H_I == 4) && (D_I == 32 || D_I == 64 || D_I == 128),
@@ -101,8 +102,10 @@ qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* 
   if (T == 0) return QSA_OK;
   REQUIRE(q_idx && w_idx && k_idx_pages && page_table && q_pos && scores, "null pointer argument");
   REQUIRE(aligned16(q_idx) && aligned16(k_idx_pages), "q_idx and k_idx_pages must be 16-byte aligned");
+  REQUIRE(aligned16(prefix_hist), "prefix_hist must be 16-byte aligned");
   qsa::IndexArgs a{q_idx, q_dt, w_idx, k_idx_pages, k_dt, num_pages, page_table, pt_rows, pt_stride,
                    q_req, q_pos, T, H_I, D_I, scores, score_stride, dev_status};
+  a.hist = prefix_hist;
   // many queries with BF16 operands (a prefill chunk): the tensor-core GEMM;
   // otherwise the streaming scan
   const cudaError_t e = (T >= 256 && qsa::index_tc_supported(a))
@@ -116,9 +119,10 @@ size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride) {
   return 0;
 }
 
-qsa_status_t qsa_topk_groups(const float* scores, int score_stride, const int32_t* q_pos, int T,
-                             int K, int32_t* sel, int32_t* n_sel, void* workspace,
-                             size_t workspace_bytes, uint32_t* dev_status, qsa_stream_t stream) {
+qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint32_t* prefix_hist,
+                             const int32_t* q_pos, int T, int K, int32_t* sel, int32_t* n_sel,
+                             void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                             qsa_stream_t stream) {
   (void)workspace; (void)workspace_bytes;
   REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
   SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
@@ -128,7 +132,9 @@ qsa_status_t qsa_topk_groups(const float* scores, int score_stride, const int32_
           score_stride, 8 * 49152);
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
+  REQUIRE(aligned16(prefix_hist), "prefix_hist must be 16-byte aligned");
   qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
+  a.hist = prefix_hist;
   return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups launch");
 }
 
@@ -145,9 +151,10 @@ qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, 
   return cuda_status(qsa::launch_expand_select(a, (cudaStream_t)stream), "qsa_expand_select launch");
 }
 
-qsa_status_t qsa_topk_expand(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,
-                             int32_t* sel, int32_t* n_sel, int32_t* tok, int32_t* n_tok, int W,
-                             uint32_t* dev_status, qsa_stream_t stream) {
+qsa_status_t qsa_topk_expand(const float* scores, int score_stride, uint32_t* prefix_hist,
+                             const int32_t* q_pos, int T, int K, int32_t* sel, int32_t* n_sel,
+                             int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
+                             qsa_stream_t stream) {
   REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
   SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
   REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
@@ -157,7 +164,9 @@ qsa_status_t qsa_topk_expand(const float* scores, int score_stride, const int32_
           score_stride, 8 * 49152);
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel && tok && n_tok, "null pointer argument");
+  REQUIRE(aligned16(prefix_hist), "prefix_hist must be 16-byte aligned");
   qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status, tok, n_tok, W};
+  a.hist = prefix_hist;
   return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_expand launch");
 }
 

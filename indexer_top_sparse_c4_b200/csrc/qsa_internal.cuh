@@ -110,6 +110,21 @@ __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// ---- score order ---------------------------------------------------------------
+// float -> uint32 whose unsigned order equals the float order; -0 maps like +0.
+// 0 is below every finite or infinite score: the Top-K uses it for "no candidate".
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t b = __float_as_uint(f);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+// Prefix histogram of a score row: counts of the top kPrefixBits bits of the
+// order keys of the row's candidate scores (QSA_PREFIX_HIST_BINS per row).
+constexpr int kPrefixBits = 12;
+constexpr int kPrefixBins = 1 << kPrefixBits;
+constexpr int kPrefixShift = 32 - kPrefixBits;
+static_assert(kPrefixBins == QSA_PREFIX_HIST_BINS, "prefix histogram width");
+
 // ---- programmatic dependent launch (PDL) ----------------------------------------
 // Every kernel of the library is launched with programmatic stream
 // serialisation, so its CTAs may be scheduled while the previous kernel on the
@@ -156,6 +171,7 @@ struct IndexArgs {
   const void* k_idx_pages; qsa_dtype_t k_dt; int num_pages;
   const int32_t* page_table; int pt_rows, pt_stride; const int32_t* q_req; const int32_t* q_pos;
   int T, H_I, D_I; float* scores; int score_stride; uint32_t* status;
+  uint32_t* hist = nullptr;  // optional [T][kPrefixBins] prefix histogram (decode scan only)
 };
 cudaError_t launch_index_scores(const IndexArgs& a, cudaStream_t s);
 // Prefill indexer on tcgen05 (BF16 query and keys, H_I = 4, D_I = 128, T >= 32)
@@ -168,6 +184,9 @@ struct TopkArgs {
   // optional: also expand the kept groups to token ids (no MTP capture);
   // tok == nullptr skips it
   int32_t* tok = nullptr; int32_t* n_tok = nullptr; int W = 0;
+  // optional [T][kPrefixBins] prefix histogram from the scan: read in place of
+  // the first cluster passes where a row's total matches, then zeroed
+  uint32_t* hist = nullptr;
 };
 int topk_cluster_size(int score_stride);       // 0: unsupported
 cudaError_t launch_topk_groups(const TopkArgs& a, cudaStream_t s);

@@ -3,25 +3,42 @@
 // exact radix Top-K is the default selector over the compressed-group
 // budget).  Ranking: score descending, ties to the lower group id.
 //
-// Design (sm_100a): one thread-block cluster of CL CTAs x 512 threads per
-// query row; thread i of CTA r owns KPT consecutive candidates in registers as
-// order-preserving uint32 keys, so the row is read from memory once (16-byte
-// loads where the row is aligned).
-//  * Radix select, 8 bits per pass from the most significant end, finds the
-//    exact key tau of the n-th largest candidate.  Each pass histograms only
-//    the keys that still match the digits found so far: per-warp shared
-//    histograms (no block-wide atomic hot spots), one block reduction, and
-//    then every CTA WRITES its 256 counts into its own slot of that pass's
-//    table in every CTA of the cluster.  After one cluster barrier each CTA
-//    adds the CL slots locally and finds the digit itself: one barrier per
-//    pass, no remote reads, no zeroing.
-//  * Output: every key > tau is kept, plus the first `need` keys == tau in
-//    index order.  Because each thread owns a contiguous run of ids, one
-//    exclusive scan over threads gives every thread the position of its first
-//    kept id within its CTA; the counts of the CTAs before it come from the
-//    histogram tables every CTA already holds (keys above tau are the keys
-//    above the chosen digit in some pass), so no further exchange is needed
-//    and the ids come out ascending with no sort.
+// Candidates become order-preserving uint32 keys; thread i of a CTA owns KPT
+// consecutive ids, so the row is read from memory once (16-byte loads where
+// the row is aligned).  Radix select over 8-bit digits from the most
+// significant end finds the exact key tau of the n-th largest candidate; the
+// output keeps every key > tau plus the first `need` keys == tau in id order.
+// Because each thread owns a contiguous run of ids, one exclusive scan over
+// the threads places every kept id, and the ids come out ascending without a
+// sort.
+//
+// Two kernels:
+//  * topk_row_kernel (many rows, e.g. a prefill chunk): one CTA per row, keys
+//    in registers, four block-local passes.  Many CTAs per SM keep the code
+//    hot in the instruction caches.
+//  * topk_cluster_kernel (few long rows, decode): one thread-block cluster of
+//    CL CTAs per row.  Each code path runs once per launch, so the kernel is
+//    written for a small instruction footprint: keys live in shared memory
+//    ([j][thread], conflict-free) and the loops over them stay rolled.
+//    - With the prefix histogram the scan built (counts of the top 12 key
+//      bits of the row), every CTA finds the 12-bit bin of the n-th largest
+//      key directly.  Each CTA lists its keys in that bin (a few hundred per
+//      row here) in its own shared memory and sends every CTA its counts in
+//      and above the bin; after one cluster barrier each CTA checks the
+//      histogram's answer against those exact counts, pulls all lists into
+//      registers with independent DSMEM loads, and finds the low 20 bits
+//      with three block-local digit passes.  A histogram that does not match
+//      (or an overfull bin) sends the row to the cluster passes below: it is
+//      a hint, and the result never depends on it.
+//    - Cluster passes: per pass, per-warp shared histograms, one block
+//      reduction, and every CTA writes its 256 counts into its own slot of
+//      that pass's table in every CTA; after one cluster barrier each CTA
+//      adds the slots and finds the digit itself.  After two passes the keys
+//      that still match the 16-bit prefix (usually a few dozen) are pushed
+//      into every CTA, which finishes the last two digits locally.
+//    - The counts of the CTAs before a CTA come from data every CTA already
+//      holds (the pass tables, or the exchanged counts), so the output needs
+//      no further exchange.
 #include <cooperative_groups.h>
 
 #include "qsa_internal.cuh"
@@ -36,27 +53,44 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;
 constexpr int kMaxCL = 8;
 
-constexpr int kCandCap = 2048;  // candidates gathered after two passes (else four cluster passes)
+constexpr int kCandCap = 2048;  // candidates gathered by a cluster (else more cluster passes)
 constexpr int kRankCap = 512;   // up to this many candidates are ranked directly
+constexpr int kKeptCap = kWarps * kBins;  // kept ids a CTA stages for its coalesced output
 
-struct TopkSmem {
+struct __align__(16) TopkSmem {
   uint32_t hw[kWarps][kBins];            // per-warp histogram of the current digit
   uint32_t hall[4][kMaxCL][kBins];       // per pass: slot q = CTA q's histogram
-  uint2 cand[kCandCap];                  // (key, id) of every candidate of the cluster
+  uint2 cand[kCandCap];                  // (key, id) candidates
   int wsum[kWarps][kMaxCL];              // block reduction of the per-CTA counts above tau
   int ccnt[2 * kMaxCL];                  // per CTA: candidates above tau, equal to tau
   int wa[kWarps];                        // per-warp scan totals
   int bin[4], above[4];
   uint32_t tau;
+  // prefix-histogram path: the bin of the n-th largest key (from the
+  // histogram), and per source CTA its keys in and above that bin
+  int pbin;
+  int scnt[kMaxCL], sgt[kMaxCL];
 };
+static_assert(kThreads * 8 == kPrefixBins, "each thread reads 8 bins of the prefix histogram");
+static_assert(sizeof(TopkSmem) % 16 == 0, "the key array after TopkSmem starts on 16 bytes");
 
-// float -> uint32 whose unsigned order equals the float order; -0 maps like +0.
-// 0 is below every finite or infinite score: it marks "no candidate".
-__device__ __forceinline__ uint32_t order_key(float f) {
-  uint32_t b = __float_as_uint(f);
-  if (b == 0x80000000u) b = 0u;
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
+// A thread's KPT keys.  RegKeys: in registers (loops over them fully
+// unrolled).  SmemKeys: in shared memory, key j of thread i at [j][i], so
+// loops over them can stay rolled (kUnroll keys per iteration).
+template <int KPT>
+struct RegKeys {
+  static constexpr int kUnroll = KPT;
+  uint32_t v[KPT];
+  __device__ __forceinline__ uint32_t get(int j) const { return v[j]; }
+  __device__ __forceinline__ void set(int j, uint32_t k) { v[j] = k; }
+};
+template <int KPT>
+struct SmemKeys {
+  static constexpr int kUnroll = 4;
+  uint32_t* col;  // this thread's column of the [KPT][kThreads] array
+  __device__ __forceinline__ uint32_t get(int j) const { return col[j * kThreads]; }
+  __device__ __forceinline__ void set(int j, uint32_t k) { col[j * kThreads] = k; }
+};
 
 template <int CL>
 __device__ __forceinline__ void csync() {
@@ -100,88 +134,212 @@ __device__ __forceinline__ void find_bin(int h, int need, int my_bin, int* bin_o
   if (lane == 31) wa[warp] = incl;
   asm volatile("bar.sync 1, %0;" ::"r"(kBins));  // the 8 warps that scan
   int above = incl - h;
-  for (int w = 0; w < warp; ++w) above += wa[w];
+#pragma unroll
+  for (int w = 0; w < kBins / 32; ++w) above += w < warp ? wa[w] : 0;
   if (above < need && above + h >= need) {
     *bin_out = my_bin;
     *above_out = above;
   }
 }
 
-template <int CL, int KPT>
-__global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int tvec) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int rank = 0;
-  if constexpr (CL > 1) rank = (int)cg::this_cluster().block_rank();
-  const int t = blockIdx.y;
-  pdl_wait();
-  const int p = a.q_pos[t];
-  int c = p >= 0 ? p / kGroupTokens : 0;
-  if (c > a.score_stride) {
-    if (rank == 0 && tid == 0) flag(a.status, QSA_DEV_ROW_RANGE);
-    c = a.score_stride;
+// CTA `rank`'s share of a row of the prefix histogram back to zero.
+template <int CL>
+__device__ __forceinline__ void zero_hist_share(uint32_t* hrow, int rank) {
+  constexpr int per = kPrefixBins / CL;
+  for (int i = rank * per + 4 * (int)threadIdx.x; i < (rank + 1) * per; i += 4 * kThreads)
+    *reinterpret_cast<uint4*>(hrow + i) = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// What a CTA knows about its row before any pass.
+struct Row {
+  int p, c, K, n;       // query position, candidates, budget, kept count
+  int cb;               // tokens of the current block (4*c(p) .. p)
+  int32_t* out;         // sel row
+  int32_t* trow;        // expanded row, or nullptr
+  uint32_t* hrow;       // prefix-histogram row, or nullptr
+};
+
+__device__ __forceinline__ Row row_of(const TopkArgs& a, int t, bool leader) {
+  Row r;
+  r.p = a.q_pos[t];
+  r.c = r.p >= 0 ? r.p / kGroupTokens : 0;
+  if (r.c > a.score_stride) {
+    if (leader) flag(a.status, QSA_DEV_ROW_RANGE);
+    r.c = a.score_stride;
   }
-  const int K = a.K;
-  const int n = c < K ? c : K;
-  int32_t* out = a.sel + (size_t)t * K;
+  r.K = a.K;
+  r.n = r.c < r.K ? r.c : r.K;
+  r.cb = r.p >= 0 ? r.p - kGroupTokens * (r.p / kGroupTokens) + 1 : 0;
+  r.out = a.sel + (size_t)t * r.K;
   // the expanded row (when asked for): 4 tokens per kept group, then the
   // current block 4*c(p) .. p, then -1
-  int32_t* trow = a.tok ? a.tok + (size_t)t * a.W : nullptr;
-  const int cb = p >= 0 ? p - kGroupTokens * (p / kGroupTokens) + 1 : 0;  // current-block tokens
-  if (c <= K) {  // every candidate is kept: dense fallback (uniform over the cluster)
-    pdl_launch_dependents();
-    for (int i = rank * kThreads + tid; i < K; i += CL * kThreads) out[i] = i < c ? i : -1;
-    if (trow) {  // tokens 0 .. p (the kept groups and the current block are contiguous)
-      const int total = kGroupTokens * n + cb;
-      for (int i = rank * kThreads + tid; i < a.W; i += CL * kThreads)
-        trow[i] = i < total ? (i < kGroupTokens * n ? i : kGroupTokens * (p / kGroupTokens) + i - kGroupTokens * n) : -1;
-      if (rank == 0 && tid == 0) {
-        a.n_tok[t] = total < a.W ? total : a.W;
-        if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
-      }
-    }
-    if (rank == 0 && tid == 0) a.n_sel[t] = n;
-    return;
-  }
+  r.trow = a.tok ? a.tok + (size_t)t * a.W : nullptr;
+  r.hrow = a.hist ? a.hist + (size_t)t * kPrefixBins : nullptr;
+  return r;
+}
 
-  // ---- this thread's KPT consecutive candidates, as keys
-  const int first = (rank * kThreads + tid) * KPT;
-  const float* row = a.scores + (size_t)t * a.score_stride;
-  uint32_t keys[KPT];
-#pragma unroll
+// c <= K: every candidate is kept (dense fallback), CTA `rank` of CL writes
+// its share of the outputs.
+template <int CL>
+__device__ __forceinline__ void dense_row(const TopkArgs& a, const Row& r, int t, int rank) {
+  const int tid = threadIdx.x;
+  if (r.hrow) zero_hist_share<CL>(r.hrow, rank);  // (not read on this path)
+  for (int i = rank * kThreads + tid; i < r.K; i += CL * kThreads) r.out[i] = i < r.c ? i : -1;
+  if (r.trow) {  // tokens 0 .. p (the kept groups and the current block are contiguous)
+    const int head = kGroupTokens * r.n, total = head + r.cb;
+    for (int i = rank * kThreads + tid; i < a.W; i += CL * kThreads)
+      r.trow[i] = i < total ? (i < head ? i : kGroupTokens * (r.p / kGroupTokens) + i - head) : -1;
+    if (rank == 0 && tid == 0) {
+      a.n_tok[t] = total < a.W ? total : a.W;
+      if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
+    }
+  }
+  if (rank == 0 && tid == 0) a.n_sel[t] = r.n;
+}
+
+// The thread's KPT consecutive candidates from `first`, as keys (0 past c).
+template <int KPT, typename Keys>
+__device__ __forceinline__ void load_keys(Keys& keys, const float* row, int first, int c, int vec) {
+  constexpr int U = Keys::kUnroll / 4 > 0 ? Keys::kUnroll / 4 : 1;
+#pragma unroll U
   for (int j = 0; j < KPT; j += 4) {
     if (vec && first + j + 3 < c) {  // 16-byte aligned when the row stride is a multiple of 4
       const float4 v = __ldg(reinterpret_cast<const float4*>(row + first + j));
-      keys[j] = order_key(v.x);
-      keys[j + 1] = order_key(v.y);
-      keys[j + 2] = order_key(v.z);
-      keys[j + 3] = order_key(v.w);
+      keys.set(j, order_key(v.x));
+      keys.set(j + 1, order_key(v.y));
+      keys.set(j + 2, order_key(v.z));
+      keys.set(j + 3, order_key(v.w));
     } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) keys[j + e] = first + j + e < c ? order_key(__ldg(row + first + j + e)) : 0u;
+      for (int e = 0; e < 4; ++e) keys.set(j + e, first + j + e < c ? order_key(__ldg(row + first + j + e)) : 0u);
     }
   }
+}
+
+// Writes this CTA's kept ids (and their tokens) at positions off ..: every
+// key > tau, and tau-keys while `rem` (those still to take at the CTA's
+// start) lasts.  gt/eq: this thread's counts; *_before: the threads' before
+// it; cta_*: the CTA's totals.  The ids are staged in shared memory (the
+// per-warp histograms, whose last use came before the block scan that gave
+// the positions) and written with coalesced stores.
+template <int KPT, typename Keys>
+__device__ __forceinline__ void emit_kept(TopkSmem& sm, const Keys& keys, int first, uint32_t tau, int gt,
+                                          int gt_before, int eq_before, int cta_gt, int cta_eq, int rem, int off,
+                                          const Row& r, int tvec) {
+  constexpr int U = Keys::kUnroll;
+  const int tid = threadIdx.x;
+  int pos = gt_before + (rem < eq_before ? rem : eq_before);  // within the CTA's kept ids
+  int take = rem - eq_before;                                 // tau-keys this thread may take
+  take = take < 0 ? 0 : take;
+  int* const kept = reinterpret_cast<int*>(&sm.hw[0][0]);
+  const int cta_kept = cta_gt + (rem < cta_eq ? rem : cta_eq);
+  const bool staged = cta_kept <= kKeptCap;  // (CTA-uniform)
+  if (gt > 0 || take > 0) {  // (most threads keep nothing)
+#pragma unroll U
+    for (int j = 0; j < KPT; ++j) {
+      const uint32_t k = keys.get(j);
+      bool keep = k > tau;
+      if (k == tau && take > 0) {
+        keep = true;
+        --take;
+      }
+      if (keep) {
+        const int g = first + j;
+        if (staged) {
+          kept[pos] = g;
+        } else if (off + pos < r.K) {
+          r.out[off + pos] = g;
+          if (r.trow) {
+#pragma unroll
+            for (int e = 0; e < kGroupTokens; ++e) r.trow[kGroupTokens * (off + pos) + e] = kGroupTokens * g + e;
+          }
+        }
+        ++pos;
+      }
+    }
+  }
+  if (staged) {
+    __syncthreads();
+    const int lim = cta_kept < r.K - off ? cta_kept : r.K - off;
+    for (int i = tid; i < lim; i += kThreads) {
+      const int g = kept[i];
+      r.out[off + i] = g;
+      if (r.trow) {
+        if (tvec) {
+          *reinterpret_cast<int4*>(r.trow + kGroupTokens * (off + i)) =
+              make_int4(kGroupTokens * g, kGroupTokens * g + 1, kGroupTokens * g + 2, kGroupTokens * g + 3);
+        } else {
+#pragma unroll
+          for (int e = 0; e < kGroupTokens; ++e) r.trow[kGroupTokens * (off + i) + e] = kGroupTokens * g + e;
+        }
+      }
+    }
+  }
+}
+
+// CTA 0's part of every row: -1 after the n kept ids, the current block and
+// the padding of the expanded row, the counts.
+__device__ __forceinline__ void write_tail(const TopkArgs& a, const Row& r, int t) {
+  const int tid = threadIdx.x;
+  for (int i = r.n + tid; i < r.K; i += kThreads) r.out[i] = -1;
+  if (tid == 0) a.n_sel[t] = r.n;
+  if (r.trow) {
+    const int head = kGroupTokens * r.n, total = head + r.cb;
+    for (int i = head + tid; i < a.W; i += kThreads)
+      r.trow[i] = i < total ? kGroupTokens * (r.p / kGroupTokens) + (i - head) : -1;
+    if (tid == 0) {
+      a.n_tok[t] = total < a.W ? total : a.W;
+      if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
+    }
+  }
+}
+
+// gt (low 16 bits) and eq (high) counts of a thread's keys against tau.
+template <int KPT, typename Keys>
+__device__ __forceinline__ int count_vs(const Keys& keys, uint32_t tau) {
+  constexpr int U = Keys::kUnroll;
+  int gt = 0, eq = 0;
+#pragma unroll U
+  for (int j = 0; j < KPT; ++j) {
+    const uint32_t k = keys.get(j);
+    gt += k > tau;
+    eq += k == tau;
+  }
+  return gt | (eq << 16);
+}
+
+// ---- many rows: one CTA per row, keys in registers --------------------------------
+template <int KPT>
+__global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int vec, int tvec) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int t = blockIdx.y;
+  pdl_wait();
+  const Row r = row_of(a, t, tid == 0);
+  if (r.c <= r.K) {
+    dense_row<1>(a, r, t, 0);
+    return;
+  }
+  if (r.hrow) zero_hist_share<1>(r.hrow, 0);  // (not read by this kernel)
+  const int first = tid * KPT;
+  RegKeys<KPT> keys;
+  load_keys<KPT>(keys, a.scores + (size_t)t * a.score_stride, first, r.c, vec);
   // (dependents launch when this grid completes: launched earlier, their CTAs
   // compete for the SMs this kernel still needs)
 
-  // ---- radix select: passes of 8 bits from the top locate tau.  After two
-  // cluster passes the keys that still match (the candidates) are usually a
-  // few dozen; then every CTA receives all of them and finishes the last two
-  // digits on its own, without further cluster barriers.
+  // ---- radix select: four passes of 8 bits from the top
   uint32_t prefix = 0;
-  int need = n;  // how many keys matching `prefix` are still to be taken
-  int npass = 4;  // cluster passes whose tables count the keys above tau
-  int ncand = 0;
+  int need = r.n;  // how many keys matching `prefix` are still to be taken
 #pragma unroll
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
 #pragma unroll
-    for (int b = lane; b < kBins; b += 32) sm.hw[warp][b] = 0u;
+    for (int b = threadIdx.x & 31; b < kBins; b += 32) sm.hw[warp][b] = 0u;
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < KPT; ++j) {
-      const uint32_t k = keys[j];
+      const uint32_t k = keys.get(j);
       const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
       if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
     }
@@ -189,53 +347,243 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
     if (tid < kBins) {
       uint32_t v = 0;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += sm.hw[w][tid];
-      if constexpr (CL > 1) {
-        cg::cluster_group cl = cg::this_cluster();
-#pragma unroll
-        for (int q = 0; q < CL; ++q) cl.map_shared_rank(&sm.hall[pass][rank][tid], q)[0] = v;
-      } else {
-        sm.hall[pass][0][tid] = v;
-      }
-    }
-    csync<CL>();  // every CTA's counts are in every CTA's table
-    if (tid < kBins) {
-      int h = 0;
-#pragma unroll
-      for (int q = 0; q < CL; ++q) h += (int)sm.hall[pass][q][kBins - 1 - tid];
-      find_bin(h, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+      for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
+      find_bin((int)v, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
     }
     __syncthreads();
     prefix |= (uint32_t)sm.bin[pass] << shift;
     need -= sm.above[pass];
-    if (CL > 1 && pass == 1) {  // (a one-CTA row keeps its four passes)
-      int total = 0;
+  }
+  const uint32_t tau = prefix;
+
+  // ---- kept ids: all keys > tau, then the first `need` keys == tau by id
+  const int ge = count_vs<KPT>(keys, tau);
+  int both;
+  const int before = block_exclusive_scan(ge, sm.wa, both);
+  emit_kept<KPT>(sm, keys, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff, both >> 16,
+                 need, 0, r, tvec);
+  write_tail(a, r, t);
+}
+
+// ---- few long rows: one cluster per row, keys in shared memory ------------------
+template <int CL, int KPT>
+__global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, int vec, int tvec) {
+  static_assert(CL > 1, "one-CTA rows use topk_row_kernel");
+  constexpr int U = SmemKeys<KPT>::kUnroll;
+  constexpr int kSeg = kCandCap / CL;           // histogram path: list capacity per CTA
+  constexpr int kSlots = kCandCap / kThreads;   // histogram path: list entries per thread
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int t = blockIdx.y;
+  pdl_wait();
+  const Row r = row_of(a, t, rank == 0 && tid == 0);
+  if (r.c <= r.K) {  // (uniform over the cluster)
+    dense_row<CL>(a, r, t, rank);
+    return;
+  }
+  const int c = r.c, n = r.n;
+
+  // ---- the prefix histogram (8 bins per thread, from the top), issued first
+  uint4 hv0 = make_uint4(0u, 0u, 0u, 0u), hv1 = hv0;
+  if (r.hrow) {
+    hv0 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 8 - 8 * tid));
+    hv1 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 4 - 8 * tid));
+  }
+  // ---- this thread's KPT consecutive candidates, as keys
+  const int first = (rank * kThreads + tid) * KPT;
+  SmemKeys<KPT> keys{reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem)) + tid};
+  load_keys<KPT>(keys, a.scores + (size_t)t * a.score_stride, first, c, vec);
+
+  uint32_t prefix = 0;
+  int need = n;    // how many keys matching `prefix` are still to be taken
+  int mode = 0;    // how tau was found: 0 four cluster passes, 1 two passes and
+                   // the gathered candidates, 2 the prefix histogram
+  int ncand = 0;
+  bool hist_zeroed = false;
+
+  if (r.hrow) {
+    // ---- the bin of the n-th largest key, from the histogram: thread tid
+    // holds bins kPrefixBins-1-8*tid-j, j = 0..7 (top first)
+    const uint32_t hb[8] = {hv1.w, hv1.z, hv1.y, hv1.x, hv0.w, hv0.z, hv0.y, hv0.x};
+    int hs = 0;
 #pragma unroll
-      for (int q = 0; q < CL; ++q) total += (int)sm.hall[1][q][sm.bin[1]];
-      if (total <= kCandCap) {  // the same decision in every CTA
-        npass = 2;
-        ncand = total;
-        break;
+    for (int j = 0; j < 8; ++j) hs += (int)hb[j];
+    int htotal;
+    const int hbefore = block_exclusive_scan(hs, sm.wa, htotal);
+    if (htotal == c) {  // (the same decision in every CTA: they read the same histogram)
+      if (hbefore < n && hbefore + hs >= n) {
+        int ab = hbefore;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (ab < n && ab + (int)hb[j] >= n) sm.pbin = kPrefixBins - 1 - 8 * tid - j;
+          ab += (int)hb[j];
+        }
+      }
+      __syncthreads();
+      const uint32_t pb = (uint32_t)sm.pbin;
+      // this CTA's keys in the bin are listed (with their ids) in its own
+      // shared memory; its counts in and above the bin go to every CTA
+      int mine = 0, above_pb = 0;
+#pragma unroll U
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t top = keys.get(j) >> kPrefixShift;
+        const bool valid = first + j < c;
+        mine += valid && top == pb;
+        above_pb += valid && top > pb;
+      }
+      int cta2;  // one scan: candidates (low 16 bits), keys above the bin (high)
+      int pos = block_exclusive_scan(mine | (above_pb << 16), sm.wa, cta2) & 0xffff;
+      if (mine) {
+#pragma unroll U
+        for (int j = 0; j < KPT; ++j) {
+          const uint32_t k = keys.get(j);
+          if (first + j < c && (k >> kPrefixShift) == pb) {
+            if (pos < kSeg) sm.cand[pos] = make_uint2(k, (uint32_t)(first + j));
+            ++pos;
+          }
+        }
+      }
+      if (tid < CL) {  // thread q tells CTA q
+        *cl.map_shared_rank(&sm.scnt[rank], tid) = cta2 & 0xffff;
+        *cl.map_shared_rank(&sm.sgt[rank], tid) = cta2 >> 16;
+      }
+      if (tid < kBins) {
+        sm.hw[0][tid] = 0u;
+        sm.hw[1][tid] = 0u;
+        sm.hw[2][tid] = 0u;
+      }
+      if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
+      csync<CL>();  // lists and counts complete; every CTA has read the histogram
+      zero_hist_share<CL>(r.hrow, rank);
+      hist_zeroed = true;
+      // the histogram's bin is taken only when the exact counts confirm it
+      int in_bin = 0, above_bin = 0;
+      bool over = false;
+#pragma unroll
+      for (int q = 0; q < CL; ++q) {
+        in_bin += sm.scnt[q];
+        above_bin += sm.sgt[q];
+        over |= sm.scnt[q] > kSeg;
+      }
+      if (!over && above_bin < n && above_bin + in_bin >= n) {
+        mode = 2;
+        need = n - above_bin;
+        prefix = pb << kPrefixShift;
+        // ---- pull every CTA's list into registers (independent DSMEM loads):
+        // slot s of thread tid is entry (tid + s*kThreads) % kSeg of CTA
+        // (tid + s*kThreads) / kSeg; then release the lists for their CTAs' exit
+        uint32_t ck[kSlots];
+        uint32_t valid = 0;
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+          const int e = tid + s * kThreads, q = e / kSeg, i = e % kSeg;
+          ck[s] = 0u;
+          if (i < sm.scnt[q]) {
+            ck[s] = cl.map_shared_rank(&sm.cand[i], q)->x;
+            valid |= 1u << s;
+          }
+        }
+        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+        // ---- the low 20 bits over the candidates: digits of 8, 8 and 4 bits
+#pragma unroll 1
+        for (int L = 0; L < 3; ++L) {
+          const int shift = L == 0 ? 12 : (L == 1 ? 4 : 0);
+          const int hi = L == 0 ? 20 : (L == 1 ? 12 : 4);  // key bits >= hi are fixed
+          const uint32_t dmask = L == 2 ? 15u : 255u;
+#pragma unroll
+          for (int s = 0; s < kSlots; ++s)
+            if (((valid >> s) & 1u) && (ck[s] >> hi) == (prefix >> hi))
+              atomicAdd(&sm.hw[L][(ck[s] >> shift) & dmask], 1u);
+          __syncthreads();
+          if (tid < kBins)
+            find_bin((int)sm.hw[L][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[L], &sm.above[L], sm.wa);
+          __syncthreads();
+          prefix |= (uint32_t)sm.bin[L] << shift;
+          need -= sm.above[L];
+        }
+        // per source CTA: candidates above and equal to tau
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s) {
+          if ((valid >> s) & 1u) {
+            const int q = (tid + s * kThreads) / kSeg;
+            if (ck[s] > prefix) atomicAdd(&sm.ccnt[q], 1);
+            else if (ck[s] == prefix) atomicAdd(&sm.ccnt[kMaxCL + q], 1);
+          }
+        }
       }
     }
   }
 
-  if constexpr (CL > 1) if (npass == 2) {
+  if (mode != 2) {
+    // ---- cluster passes of 8 bits from the top.  After two, the keys that
+    // still match (the candidates) are usually a few dozen; then every CTA
+    // receives all of them and finishes the last two digits on its own.
+    mode = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+#pragma unroll
+      for (int b = lane; b < kBins; b += 32) sm.hw[warp][b] = 0u;
+      __syncwarp();
+#pragma unroll U
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t k = keys.get(j);
+        const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
+        if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
+      }
+      __syncthreads();
+      if (tid < kBins) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += sm.hw[w][tid];
+#pragma unroll
+        for (int q = 0; q < CL; ++q) cl.map_shared_rank(&sm.hall[pass][rank][tid], q)[0] = v;
+      }
+      csync<CL>();  // every CTA's counts are in every CTA's table
+      if (pass == 0 && r.hrow && !hist_zeroed) zero_hist_share<CL>(r.hrow, rank);
+      if (tid < kBins) {
+        int h = 0;
+#pragma unroll
+        for (int q = 0; q < CL; ++q) h += (int)sm.hall[pass][q][kBins - 1 - tid];
+        find_bin(h, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sm.bin[pass] << shift;
+      need -= sm.above[pass];
+      if (pass == 1) {
+        int total = 0;
+#pragma unroll
+        for (int q = 0; q < CL; ++q) total += (int)sm.hall[1][q][sm.bin[1]];
+        if (total <= kCandCap) {  // the same decision in every CTA
+          mode = 1;
+          ncand = total;
+          break;
+        }
+      }
+    }
+  }
+
+  if (mode == 1) {
     // ---- candidates: every CTA writes its keys matching the 16-bit prefix,
     // with their ids, into every CTA's list (CTA q's block starts after the
     // candidates of CTAs 0 .. q-1, whose counts pass 1's table holds)
     int mine = 0;
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) mine += (keys[j] >> 16) == (prefix >> 16);
+#pragma unroll U
+    for (int j = 0; j < KPT; ++j) mine += (keys.get(j) >> 16) == (prefix >> 16);
     int cta_total;
     int pos = block_exclusive_scan(mine, sm.wa, cta_total);
-    for (int q = 0; q < rank; ++q) pos += (int)sm.hall[1][q][sm.bin[1]];
-    if (mine) {
-      cg::cluster_group cl = cg::this_cluster();
 #pragma unroll
+    for (int q = 0; q < CL; ++q) pos += q < rank ? (int)sm.hall[1][q][sm.bin[1]] : 0;
+    if (mine) {
+#pragma unroll U
       for (int j = 0; j < KPT; ++j) {
-        if ((keys[j] >> 16) == (prefix >> 16)) {
-          const uint2 e = make_uint2(keys[j], (uint32_t)(first + j));
+        const uint32_t k = keys.get(j);
+        if ((k >> 16) == (prefix >> 16)) {
+          const uint2 e = make_uint2(k, (uint32_t)(first + j));
+#pragma unroll
           for (int q = 0; q < CL; ++q) *cl.map_shared_rank(&sm.cand[pos], q) = e;
           ++pos;
         }
@@ -248,13 +596,13 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
       // direct count; the candidate of rank need-1 is tau
       if (tid < ncand) {
         const uint2 me = sm.cand[tid];
-        int r = 0, r_key = 0;  // rank, and candidates with a larger key
+        int rk = 0, r_key = 0;  // rank, and candidates with a larger key
         for (int i = 0; i < ncand; ++i) {
           const uint2 o = sm.cand[i];
-          r += o.x > me.x || (o.x == me.x && o.y < me.y);
+          rk += o.x > me.x || (o.x == me.x && o.y < me.y);
           r_key += o.x > me.x;
         }
-        if (r == need - 1) {
+        if (rk == need - 1) {
           sm.tau = me.x;
           sm.above[2] = r_key;  // candidates above tau
         }
@@ -264,7 +612,7 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
       need -= sm.above[2];
     } else {
       // ---- the last two digits, over the candidates only
-#pragma unroll
+#pragma unroll 1
       for (int pass = 2; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         if (tid < kBins) sm.hw[0][tid] = 0u;
@@ -291,12 +639,13 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
   }
   const uint32_t tau = prefix;
 
-  // ---- keys above tau in each CTA: a key is above tau when, in the first
-  // pass where its digit differs from tau's, its digit is the larger one, and
-  // that pass's table counted it under that digit in its CTA's slot (on the
-  // candidate path the last two passes are counted from the candidate list)
-  if (tid < kBins) {
-    int x[kMaxCL];
+  // ---- keys above tau in each CTA, on the table paths: a key is above tau
+  // when, in the first pass where its digit differs from tau's, its digit is
+  // the larger one, and that pass's table counted it under that digit in its
+  // CTA's slot (after two passes the candidate list counts the rest)
+  if (mode != 2 && tid < kBins) {
+    const int npass = mode == 1 ? 2 : 4;
+    int x[CL];
 #pragma unroll
     for (int q = 0; q < CL; ++q) x[q] = 0;
 #pragma unroll
@@ -315,97 +664,64 @@ __global__ void __launch_bounds__(kThreads) topk_kernel(TopkArgs a, int vec, int
   }
 
   // ---- kept ids: all keys > tau, then the first `need` keys == tau by id
-  int gt = 0, eq = 0;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    gt += keys[j] > tau;
-    eq += keys[j] == tau;
-  }
-  int both;  // one scan of gt (low 16 bits) and eq (high): per-CTA counts stay below 2^16
-  const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum, ccnt visible
-  const int gt_before = before & 0xffff, eq_before = before >> 16;
+  const int ge = count_vs<KPT>(keys, tau);
+  int both;  // per-CTA counts stay below 2^16
+  const int before = block_exclusive_scan(ge, sm.wa, both);  // syncs: wsum, ccnt visible
   // the CTAs before this one: lane q of every warp takes CTA q's counts, and a
   // warp prefix over q gives the offsets (no serial loop, no extra barrier)
-  int off = 0, eq_prev = 0;
-  if constexpr (CL > 1) {
-    int gt_q = 0, eq_q = 0;
-    if (lane < CL) {
-      gt_q = npass == 2 ? sm.ccnt[lane] : 0;
+  int gt_q = 0, eq_q = 0;
+  if (lane < CL) {
+    if (mode == 2) {  // keys above the bin, plus candidates above tau
+      gt_q = sm.sgt[lane] + sm.ccnt[lane];
+      eq_q = sm.ccnt[kMaxCL + lane];
+    } else {
+      gt_q = mode == 1 ? sm.ccnt[lane] : 0;
 #pragma unroll
       for (int w = 0; w < kBins / 32; ++w) gt_q += sm.wsum[w][lane];
-      eq_q = npass == 2 ? sm.ccnt[kMaxCL + lane] : (int)sm.hall[3][lane][sm.bin[3]];
+      eq_q = mode == 1 ? sm.ccnt[kMaxCL + lane] : (int)sm.hall[3][lane][sm.bin[3]];
     }
-    // exclusive prefix over lanes q < rank of the kept count: gt_q plus the
-    // tau-keys CTA q takes, which depends on the tau-keys before it
-    int eq_incl = eq_q;
-#pragma unroll
-    for (int d = 1; d < kMaxCL; d <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, eq_incl, d);
-      if (lane >= d) eq_incl += u;
-    }
-    const int eq_before_q = eq_incl - eq_q;
-    const int rem_q = need - eq_before_q;
-    int kept_q = lane < rank ? gt_q + (rem_q <= 0 ? 0 : (rem_q < eq_q ? rem_q : eq_q)) : 0;
-#pragma unroll
-    for (int d = 1; d < kMaxCL; d <<= 1) kept_q += __shfl_xor_sync(0xffffffffu, kept_q, d);
-    off = __shfl_sync(0xffffffffu, kept_q, 0);
-    eq_prev = __shfl_sync(0xffffffffu, eq_before_q, rank);
   }
-  int rem = need - eq_prev;                     // tau-keys still to take at this CTA's start
+  // exclusive prefix over lanes q < rank of the kept count: gt_q plus the
+  // tau-keys CTA q takes, which depends on the tau-keys before it
+  int eq_incl = eq_q;
+#pragma unroll
+  for (int d = 1; d < kMaxCL; d <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, eq_incl, d);
+    if (lane >= d) eq_incl += u;
+  }
+  const int eq_before_q = eq_incl - eq_q;
+  const int rem_q = need - eq_before_q;
+  int kept_q = lane < rank ? gt_q + (rem_q <= 0 ? 0 : (rem_q < eq_q ? rem_q : eq_q)) : 0;
+#pragma unroll
+  for (int d = 1; d < kMaxCL; d <<= 1) kept_q += __shfl_xor_sync(0xffffffffu, kept_q, d);
+  const int off = __shfl_sync(0xffffffffu, kept_q, 0);
+  const int eq_prev = __shfl_sync(0xffffffffu, eq_before_q, rank);
+  int rem = need - eq_prev;  // tau-keys still to take at this CTA's start
   rem = rem < 0 ? 0 : rem;
-  int pos = off + gt_before + (rem < eq_before ? rem : eq_before);
-  int take = rem - eq_before;                   // tau-keys this thread may take
-  take = take < 0 ? 0 : take;
-  if (gt > 0 || take > 0)  // (most threads keep nothing)
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const uint32_t k = keys[j];
-    bool keep = k > tau;
-    if (k == tau && take > 0) {
-      keep = true;
-      --take;
-    }
-    if (keep) {
-      if (pos < K) {
-        const int g = first + j;
-        out[pos] = g;
-        if (trow) {
-          if (tvec) {
-            *reinterpret_cast<int4*>(trow + kGroupTokens * pos) =
-                make_int4(kGroupTokens * g, kGroupTokens * g + 1, kGroupTokens * g + 2, kGroupTokens * g + 3);
-          } else {
-#pragma unroll
-            for (int e = 0; e < kGroupTokens; ++e) trow[kGroupTokens * pos + e] = kGroupTokens * g + e;
-          }
-        }
-      }
-      ++pos;
-    }
-  }
-  if (rank == 0) {
-    for (int i = n + tid; i < K; i += kThreads) out[i] = -1;
-    if (tid == 0) a.n_sel[t] = n;
-    if (trow) {  // the current block, then padding
-      const int head = kGroupTokens * n, total = head + cb;
-      for (int i = head + tid; i < a.W; i += kThreads)
-        trow[i] = i < total ? kGroupTokens * (p / kGroupTokens) + (i - head) : -1;
-      if (tid == 0) {
-        a.n_tok[t] = total < a.W ? total : a.W;
-        if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
-      }
-    }
-  }
+  emit_kept<KPT>(sm, keys, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff, both >> 16,
+                 rem, off, r, tvec);
+  if (rank == 0) write_tail(a, r, t);
+  // the other CTAs read this CTA's candidate list: stay until they have
+  if (mode == 2) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <int CL, int KPT>
 cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
-  const size_t smem = sizeof(TopkSmem);
-  auto kern = topk_kernel<CL, KPT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   const int vec = (a.score_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
   const int tvec = a.tok && a.W % 4 == 0 && (reinterpret_cast<uintptr_t>(a.tok) & 15u) == 0;
-  return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec, tvec);
+  if constexpr (CL == 1) {
+    const size_t smem = sizeof(TopkSmem);
+    auto kern = topk_row_kernel<KPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(1, a.T), dim3(kThreads), smem, s, 1, a, vec, tvec);
+  } else {
+    const size_t smem = sizeof(TopkSmem) + (size_t)KPT * kThreads * sizeof(uint32_t);
+    auto kern = topk_cluster_kernel<CL, KPT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec, tvec);
+  }
 }
 
 template <int KPT>

@@ -20,7 +20,7 @@ from .workloads import GROUP_TOKENS, Workload
 
 class QSAStep:
     def __init__(self, w: Workload, prefill: bool | None = None, out_dtype=None,
-                 score_stride: int | None = None):
+                 score_stride: int | None = None, prefix_hist: bool | None = None):
         self.w = w
         dev = w.q.device
         self.prefill = (w.T > 64) if prefill is None else prefill
@@ -47,16 +47,24 @@ class QSAStep:
         self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
         tk = qsa.qsa_topk_groups_workspace_size(T, w.K, self.score_stride)
         self.topk_ws = torch.empty((max(tk, 16),), dtype=torch.uint8, device=dev) if tk else None
+        # the scan's 12-bit key-prefix counts, handed to the Top-K (decode rows);
+        # zero at allocation, and every Top-K call leaves it zero again
+        if prefix_hist is None:
+            prefix_hist = not self.prefill
+        self.prefix_hist = (torch.zeros((T, qsa.QSA_PREFIX_HIST_BINS), dtype=torch.int32, device=dev)
+                            if prefix_hist else None)
 
     # the four stages, separately callable for per-stage tests and timing
     def index_scores(self, stream=None):
         w = self.w
         qsa.qsa_index_scores(w.q_idx, w.w_idx, w.k_idx_pages, w.page_table, self.sel_pos,
-                             self.scores, q_req=w.q_req, dev_status=self.status, stream=stream)
+                             self.scores, q_req=w.q_req, dev_status=self.status, stream=stream,
+                             prefix_hist=self.prefix_hist)
 
     def topk(self, stream=None):
         qsa.qsa_topk_groups(self.scores, self.sel_pos, self.w.K, self.sel, self.n_sel,
-                            workspace=self.topk_ws, dev_status=self.status, stream=stream)
+                            workspace=self.topk_ws, dev_status=self.status, stream=stream,
+                            prefix_hist=self.prefix_hist)
 
     def expand(self, stream=None):
         w = self.w
@@ -79,7 +87,7 @@ class QSAStep:
         w = self.w
         if w.capture_pos is None:
             qsa.qsa_topk_expand(self.scores, w.q_pos, w.K, self.sel, self.n_sel, self.tok, self.n_tok,
-                                dev_status=self.status, stream=stream)
+                                dev_status=self.status, stream=stream, prefix_hist=self.prefix_hist)
         else:
             self.topk(stream)
             self.expand(stream)

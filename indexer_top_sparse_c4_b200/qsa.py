@@ -21,6 +21,7 @@ QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUD
 QSA_F32, QSA_BF16, QSA_FP8_E4M3 = 0, 1, 2
 QSA_DEV_BAD_PAGE, QSA_DEV_BAD_TOKEN, QSA_DEV_BAD_GROUP, QSA_DEV_ROW_RANGE = 1, 2, 4, 8
 QSA_DEV_BAD_REQUEST, QSA_DEV_TIMEOUT = 16, 32
+QSA_PREFIX_HIST_BINS = 4096
 
 ENTRY_POINTS = (
     "qsa_index_scores", "qsa_topk_groups_workspace_size", "qsa_topk_groups",
@@ -49,12 +50,12 @@ def lib() -> ctypes.CDLL:
                            "`python -m indexer_top_sparse_c4_b200.build` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    L.qsa_index_scores.argtypes = [P, I, P, P, I, I, P, I, I, P, P, I, I, I, P, I, P, P]
+    L.qsa_index_scores.argtypes = [P, I, P, P, I, I, P, I, I, P, P, I, I, I, P, I, P, P, P]
     L.qsa_topk_groups_workspace_size.argtypes = [I, I, I]
     L.qsa_topk_groups_workspace_size.restype = U
-    L.qsa_topk_groups.argtypes = [P, I, P, I, I, P, P, P, U, P, P]
+    L.qsa_topk_groups.argtypes = [P, I, P, P, I, I, P, P, P, U, P, P]
     L.qsa_expand_select.argtypes = [P, P, I, P, P, I, P, P, I, P, P]
-    L.qsa_topk_expand.argtypes = [P, I, P, I, I, P, P, P, P, I, P, P]
+    L.qsa_topk_expand.argtypes = [P, I, P, P, I, I, P, P, P, P, I, P, P]
     L.qsa_sparse_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
     L.qsa_sparse_attn_decode_workspace_size.restype = U
     L.qsa_sparse_attn_decode.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
@@ -109,13 +110,16 @@ def _stream(stream) -> ctypes.c_void_p:
 
 
 def qsa_index_scores(q_idx, w_idx, k_idx_pages, page_table, q_pos, scores, q_req=None,
-                     dev_status=None, stream=None):
+                     dev_status=None, stream=None, prefix_hist=None):
+    """prefix_hist: optional int32/uint32 [T, QSA_PREFIX_HIST_BINS], zero on
+    entry; receives the row's 12-bit key-prefix counts (see qsa.h)."""
     T, H_I, D_I = q_idx.shape
     _check(lib().qsa_index_scores(
         _ptr(q_idx), _dt(q_idx), _ptr(w_idx), _ptr(k_idx_pages), _dt(k_idx_pages),
         k_idx_pages.shape[0], _ptr(page_table), page_table.shape[0], page_table.shape[1],
         _ptr(q_req), _ptr(q_pos),
-        T, H_I, D_I, _ptr(scores), scores.shape[1], _ptr(dev_status), _stream(stream)))
+        T, H_I, D_I, _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(dev_status),
+        _stream(stream)))
     return scores
 
 
@@ -123,12 +127,13 @@ def qsa_topk_groups_workspace_size(T, K, score_stride) -> int:
     return int(lib().qsa_topk_groups_workspace_size(T, K, score_stride))
 
 
-def qsa_topk_groups(scores, q_pos, K, sel, n_sel, workspace=None, dev_status=None, stream=None):
+def qsa_topk_groups(scores, q_pos, K, sel, n_sel, workspace=None, dev_status=None, stream=None,
+                    prefix_hist=None):
     T = scores.shape[0]
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().qsa_topk_groups(
-        _ptr(scores), scores.shape[1], _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel), _ptr(workspace),
-        ws_bytes, _ptr(dev_status), _stream(stream)))
+        _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel),
+        _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
     return sel, n_sel
 
 
@@ -140,12 +145,13 @@ def qsa_expand_select(sel, n_sel, q_pos, tok, n_tok, capture_pos=None, dev_statu
     return tok, n_tok
 
 
-def qsa_topk_expand(scores, q_pos, K, sel, n_sel, tok, n_tok, dev_status=None, stream=None):
+def qsa_topk_expand(scores, q_pos, K, sel, n_sel, tok, n_tok, dev_status=None, stream=None,
+                    prefix_hist=None):
     """Top-K and expansion in one launch (rows without an MTP capture)."""
     T, score_stride = scores.shape
     _check(lib().qsa_topk_expand(
-        _ptr(scores), score_stride, _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel), _ptr(tok),
-        _ptr(n_tok), tok.shape[1], _ptr(dev_status), _stream(stream)))
+        _ptr(scores), score_stride, _ptr(prefix_hist), _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel),
+        _ptr(tok), _ptr(n_tok), tok.shape[1], _ptr(dev_status), _stream(stream)))
     return sel, n_sel, tok, n_tok
 
 

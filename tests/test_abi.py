@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 3
+    assert L.qsa_abi_version() == 4
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -57,30 +57,41 @@ NULL = None
 
 
 def test_index_scores_rejects_unbuilt_shapes(L):
-    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 3, 128, NULL, 16, NULL, NULL)
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 3, 128, NULL, 16, NULL, NULL, NULL)
     assert st == 2 and "H_I" in _err(L)
-    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, -1, 4, 128, NULL, 16, NULL, NULL)
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, -1, 4, 128, NULL, 16, NULL, NULL, NULL)
     assert st == 1
-    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL)
+    st = L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL, NULL)
     assert st == 1 and "null" in _err(L)
-    st = L.qsa_index_scores(NULL, 2, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL)
+    st = L.qsa_index_scores(NULL, 2, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 4, 4, 128, NULL, 16, NULL, NULL, NULL)
     assert st == 1 and "dtype" in _err(L)
     # T == 0 is a no-op that launches nothing
-    assert L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 0, 4, 128, NULL, 16, NULL, NULL) == 0
+    assert L.qsa_index_scores(NULL, 0, NULL, NULL, 0, 1, NULL, 1, 1, NULL, NULL, 0, 4, 128, NULL, 16, NULL, NULL, NULL) == 0
 
 
 def test_index_scores_rejects_misaligned_pointers(L):
     bad = ctypes.c_void_p(0x1004)
     ok = ctypes.c_void_p(0x2000)
-    st = L.qsa_index_scores(bad, 0, ok, ok, 0, 1, ok, 1, 1, NULL, ok, 1, 4, 128, ok, 16, NULL, NULL)
+    st = L.qsa_index_scores(bad, 0, ok, ok, 0, 1, ok, 1, 1, NULL, ok, 1, 4, 128, ok, 16, NULL, NULL, NULL)
     assert st == 1 and "aligned" in _err(L)
 
 
+def test_prefix_hist_must_be_aligned(L):
+    ok = ctypes.c_void_p(0x2000)
+    bad = ctypes.c_void_p(0x2008)
+    st = L.qsa_index_scores(ok, 0, ok, ok, 0, 1, ok, 1, 1, NULL, ok, 1, 4, 128, ok, 16, bad, NULL, NULL)
+    assert st == 1 and "prefix_hist" in _err(L)
+    assert L.qsa_topk_groups(ok, 16, bad, ok, 1, 4, ok, ok, NULL, 0, NULL, NULL) == 1
+    assert "prefix_hist" in _err(L)
+    assert L.qsa_topk_expand(ok, 16, bad, ok, 1, 4, ok, ok, ok, ok, 20, NULL, NULL) == 1
+    assert "prefix_hist" in _err(L)
+
+
 def test_topk_validation(L):
-    assert L.qsa_topk_groups(NULL, 16, NULL, 2, 0, NULL, NULL, NULL, 0, NULL, NULL) == 1
-    assert L.qsa_topk_groups(NULL, 0, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 1
-    assert L.qsa_topk_groups(NULL, 10 ** 7, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 2
-    assert L.qsa_topk_groups(NULL, 16, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 0
+    assert L.qsa_topk_groups(NULL, 16, NULL, NULL, 2, 0, NULL, NULL, NULL, 0, NULL, NULL) == 1
+    assert L.qsa_topk_groups(NULL, 0, NULL, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 1
+    assert L.qsa_topk_groups(NULL, 10 ** 7, NULL, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 2
+    assert L.qsa_topk_groups(NULL, 16, NULL, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 0
     assert L.qsa_topk_groups_workspace_size(8, 512, 65535) == 0
 
 
@@ -92,14 +103,14 @@ def test_expand_validation(L):
 
 
 def test_topk_expand_validation(L):
-    # (scores, stride, q_pos, T, K, sel, n_sel, tok, n_tok, W, status, stream)
-    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 8, NULL, NULL, NULL, NULL, 35, NULL, NULL) == 1
+    # (scores, stride, prefix_hist, q_pos, T, K, sel, n_sel, tok, n_tok, W, status, stream)
+    assert L.qsa_topk_expand(NULL, 16, NULL, NULL, 1, 8, NULL, NULL, NULL, NULL, 35, NULL, NULL) == 1
     assert "4*K + 4" in _err(L)
-    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 0, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
-    assert L.qsa_topk_expand(NULL, 10 ** 7, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 2
-    assert L.qsa_topk_expand(NULL, 16, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
+    assert L.qsa_topk_expand(NULL, 16, NULL, NULL, 1, 0, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
+    assert L.qsa_topk_expand(NULL, 10 ** 7, NULL, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 2
+    assert L.qsa_topk_expand(NULL, 16, NULL, NULL, 1, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 1
     assert "null" in _err(L)
-    assert L.qsa_topk_expand(NULL, 16, NULL, 0, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 0
+    assert L.qsa_topk_expand(NULL, 16, NULL, NULL, 0, 8, NULL, NULL, NULL, NULL, 36, NULL, NULL) == 0
 
 
 def _attn(L, fn, T=1, Hq=16, Hkv=2, D=256, kv_dt=1, q_dt=1, out_dt=1, W=36, ks=1.0, vs=1.0,

@@ -213,6 +213,96 @@ def test_topk_expand_matches_separate_calls(case):
         assert torch.equal(x, y)
 
 
+def _host_prefix_hist(scores, q_pos, stride):
+    """Per row: counts of the top 12 bits of the order keys of the candidate
+    scores, computed on the host from the GPU's own scores."""
+    b = np.ascontiguousarray(scores).view(np.uint32).copy()
+    b[b == 0x80000000] = 0
+    key = np.where(b & 0x80000000, ~b, b | 0x80000000).astype(np.uint32)
+    out = np.zeros((scores.shape[0], 4096), np.int64)
+    for t in range(scores.shape[0]):
+        c = min(max(int(q_pos[t]), 0) // 4, stride)
+        out[t] = np.bincount(key[t, :c] >> 20, minlength=4096)
+    return out
+
+
+def _fake_hist(scores, q_pos, stride, how):
+    """A histogram that sums to each row's candidate count but is wrong."""
+    h = np.zeros((scores.shape[0], 4096), np.int32)
+    true = _host_prefix_hist(scores, q_pos, stride)
+    for t in range(scores.shape[0]):
+        c = int(true[t].sum())
+        nz = np.nonzero(true[t])[0]
+        if how == "one_bin":       # every count in the row's highest occupied bin
+            h[t, nz.max()] = c
+        else:                      # the true counts moved one bin up
+            h[t, np.minimum(nz + 1, 4095)] += true[t, nz].astype(np.int32)
+    return h
+
+
+@pytest.mark.parametrize("case", ["b1_16k", "b4_65k_peaked", "b2_262k_peaked", "b2_65k_normal_k2048",
+                                  "ties", "tiny", "dense_fallback"])
+def test_prefix_hist(case):
+    """The scan's prefix histogram equals the one counted on the host from its
+    scores; the Top-K (and the fused expansion) given it returns exactly what
+    it returns without it, and leaves it zero.  A wrong histogram that still
+    sums to the candidate count (every count in one bin; counts moved one bin
+    up) changes nothing either: the kernel checks the histogram's bin against
+    exact counts before using it."""
+    from indexer_top_sparse_c4_b200 import qsa
+    if case == "b1_16k":
+        w = wl.b1_16k(device="cuda")
+    elif case == "b4_65k_peaked":      # clusters of 2 CTAs per row
+        w = wl.b8_262k(device="cuda", B=4, ctx=65536)
+    elif case == "b2_262k_peaked":     # clusters of 8 CTAs per row
+        w = wl.b8_262k(device="cuda", B=2)
+    elif case == "b2_65k_normal_k2048":
+        w = wl.b8_262k(device="cuda", B=2, ctx=65536, K=2048, dist="normal", kv_dtype="bf16")
+    elif case == "ties":   # 16 score levels: the tie bins overflow the candidate lists
+        w = wl.b8_262k(device="cuda", B=2, ctx=65536, dist="ties")
+    elif case == "tiny":
+        w = wl.tiny(device="cuda")
+    else:
+        w = wl.b1_16k(device="cuda", K=8192)
+    step = QSAStep(w, prefix_hist=True)
+    step.index_scores()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    scores = host(step.scores)
+    q_pos = host(w.q_pos)
+    want = _host_prefix_hist(scores, q_pos, step.score_stride)
+    got = host(step.prefix_hist).astype(np.int64)
+    assert np.array_equal(got, want)
+    saved = step.prefix_hist.clone()
+    T, K, W = w.T, w.K, w.W
+
+    def run(hist, fused):
+        sel = torch.full((T, K), 7, dtype=torch.int32, device="cuda")
+        n_sel = torch.full((T,), 7, dtype=torch.int32, device="cuda")
+        tok = torch.full((T, W), 7, dtype=torch.int32, device="cuda")
+        n_tok = torch.full((T,), 7, dtype=torch.int32, device="cuda")
+        status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        if fused:
+            qsa.qsa_topk_expand(step.scores, w.q_pos, K, sel, n_sel, tok, n_tok, dev_status=status,
+                                prefix_hist=hist)
+        else:
+            qsa.qsa_topk_groups(step.scores, w.q_pos, K, sel, n_sel, dev_status=status, prefix_hist=hist)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        return (sel, n_sel, tok, n_tok) if fused else (sel, n_sel)
+
+    for fused in (False, True):
+        ref = run(None, fused)
+        hists = [saved.clone(),
+                 torch.from_numpy(_fake_hist(scores, q_pos, step.score_stride, "one_bin")).cuda(),
+                 torch.from_numpy(_fake_hist(scores, q_pos, step.score_stride, "shifted")).cuda()]
+        for h in hists:
+            got = run(h, fused)
+            for x, y in zip(ref, got):
+                assert torch.equal(x, y)
+            assert int(torch.count_nonzero(h).item()) == 0
+
+
 def test_mtp_draft_reuse(oracle):
     w = wl.mtp(device="cuda")
     step = QSAStep(w)
