@@ -70,6 +70,8 @@ struct __align__(16) TopkSmem {
   // histogram), and per source CTA its keys in and above that bin
   int pbin;
   int scnt[kMaxCL], sgt[kMaxCL];
+  uint2 fin[kRankCap];                   // candidates left after the first local digit
+  int nfin;
 };
 static_assert(kThreads * 8 == kPrefixBins, "each thread reads 8 bins of the prefix histogram");
 static_assert(sizeof(TopkSmem) % 16 == 0, "the key array after TopkSmem starts on 16 bytes");
@@ -219,13 +221,15 @@ __device__ __forceinline__ void load_keys(Keys& keys, const float* row, int firs
 // Writes this CTA's kept ids (and their tokens) at positions off ..: every
 // key > tau, and tau-keys while `rem` (those still to take at the CTA's
 // start) lasts.  gt/eq: this thread's counts; *_before: the threads' before
-// it; cta_*: the CTA's totals.  The ids are staged in shared memory (the
-// per-warp histograms, whose last use came before the block scan that gave
-// the positions) and written with coalesced stores.
-template <int KPT, typename Keys>
-__device__ __forceinline__ void emit_kept(TopkSmem& sm, const Keys& keys, int first, uint32_t tau, int gt,
-                                          int gt_before, int eq_before, int cta_gt, int cta_eq, int rem, int off,
-                                          const Row& r, int tvec) {
+// it; cta_*: the CTA's totals.  MASKED: only the keys flagged in above_mask
+// (certainly kept) and cand_mask (compared with tau) are visited; otherwise
+// all KPT.  The ids are staged in shared memory (the per-warp histograms,
+// whose last use came before the block scan that gave the positions) and
+// written with coalesced stores.
+template <int KPT, bool MASKED, typename Keys>
+__device__ __forceinline__ void emit_kept(TopkSmem& sm, const Keys& keys, uint64_t above_mask, uint64_t cand_mask,
+                                          int first, uint32_t tau, int gt, int gt_before, int eq_before, int cta_gt,
+                                          int cta_eq, int rem, int off, const Row& r, int tvec) {
   constexpr int U = Keys::kUnroll;
   const int tid = threadIdx.x;
   int pos = gt_before + (rem < eq_before ? rem : eq_before);  // within the CTA's kept ids
@@ -234,28 +238,39 @@ __device__ __forceinline__ void emit_kept(TopkSmem& sm, const Keys& keys, int fi
   int* const kept = reinterpret_cast<int*>(&sm.hw[0][0]);
   const int cta_kept = cta_gt + (rem < cta_eq ? rem : cta_eq);
   const bool staged = cta_kept <= kKeptCap;  // (CTA-uniform)
-  if (gt > 0 || take > 0) {  // (most threads keep nothing)
-#pragma unroll U
-    for (int j = 0; j < KPT; ++j) {
+  auto visit = [&](int j, bool above) {
+    bool keep = above;
+    if (!above) {
       const uint32_t k = keys.get(j);
-      bool keep = k > tau;
+      keep = k > tau;
       if (k == tau && take > 0) {
         keep = true;
         --take;
       }
-      if (keep) {
-        const int g = first + j;
-        if (staged) {
-          kept[pos] = g;
-        } else if (off + pos < r.K) {
-          r.out[off + pos] = g;
-          if (r.trow) {
+    }
+    if (keep) {
+      const int g = first + j;
+      if (staged) {
+        kept[pos] = g;
+      } else if (off + pos < r.K) {
+        r.out[off + pos] = g;
+        if (r.trow) {
 #pragma unroll
-            for (int e = 0; e < kGroupTokens; ++e) r.trow[kGroupTokens * (off + pos) + e] = kGroupTokens * g + e;
-          }
+          for (int e = 0; e < kGroupTokens; ++e) r.trow[kGroupTokens * (off + pos) + e] = kGroupTokens * g + e;
         }
-        ++pos;
       }
+      ++pos;
+    }
+  };
+  if (gt > 0 || take > 0) {  // (most threads keep nothing)
+    if constexpr (MASKED) {
+      for (uint64_t m = above_mask | cand_mask; m; m &= m - 1) {
+        const int j = __ffsll((long long)m) - 1;
+        visit(j, (above_mask >> j) & 1u);
+      }
+    } else {
+#pragma unroll U
+      for (int j = 0; j < KPT; ++j) visit(j, false);
     }
   }
   if (staged) {
@@ -360,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
   const int ge = count_vs<KPT>(keys, tau);
   int both;
   const int before = block_exclusive_scan(ge, sm.wa, both);
-  emit_kept<KPT>(sm, keys, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff, both >> 16,
-                 need, 0, r, tvec);
+  emit_kept<KPT, false>(sm, keys, 0, 0, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff,
+                        both >> 16, need, 0, r, tvec);
   write_tail(a, r, t);
 }
 
@@ -369,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
 template <int CL, int KPT>
 __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, int vec, int tvec) {
   static_assert(CL > 1, "one-CTA rows use topk_row_kernel");
+  static_assert(KPT <= 64, "key masks are 64 bits");
   constexpr int U = SmemKeys<KPT>::kUnroll;
   constexpr int kSeg = kCandCap / CL;           // histogram path: list capacity per CTA
   constexpr int kSlots = kCandCap / kThreads;   // histogram path: list entries per thread
@@ -386,34 +402,41 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
   }
   const int c = r.c, n = r.n;
 
-  // ---- the prefix histogram (8 bins per thread, from the top), issued first
+  // ---- loads: the prefix histogram (8 bins per thread, from the top) and
+  // this thread's KPT consecutive scores
   uint4 hv0 = make_uint4(0u, 0u, 0u, 0u), hv1 = hv0;
   if (r.hrow) {
     hv0 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 8 - 8 * tid));
     hv1 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 4 - 8 * tid));
   }
-  // ---- this thread's KPT consecutive candidates, as keys
   const int first = (rank * kThreads + tid) * KPT;
-  SmemKeys<KPT> keys{reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem)) + tid};
-  load_keys<KPT>(keys, a.scores + (size_t)t * a.score_stride, first, c, vec);
+  const float* row = a.scores + (size_t)t * a.score_stride;
+  float sc[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; j += 4) {
+    if (vec && first + j + 3 < c) {  // 16-byte aligned when the row stride is a multiple of 4
+      const float4 v = __ldg(reinterpret_cast<const float4*>(row + first + j));
+      sc[j] = v.x;
+      sc[j + 1] = v.y;
+      sc[j + 2] = v.z;
+      sc[j + 3] = v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sc[j + e] = first + j + e < c ? __ldg(row + first + j + e) : 0.f;
+    }
+  }
 
-  uint32_t prefix = 0;
-  int need = n;    // how many keys matching `prefix` are still to be taken
-  int mode = 0;    // how tau was found: 0 four cluster passes, 1 two passes and
-                   // the gathered candidates, 2 the prefix histogram
-  int ncand = 0;
-  bool hist_zeroed = false;
-
+  // ---- the bin of the n-th largest key, from the histogram
+  bool hist_ok = false;  // (the same in every CTA: they read the same histogram)
+  uint32_t pb = 0;
   if (r.hrow) {
-    // ---- the bin of the n-th largest key, from the histogram: thread tid
-    // holds bins kPrefixBins-1-8*tid-j, j = 0..7 (top first)
     const uint32_t hb[8] = {hv1.w, hv1.z, hv1.y, hv1.x, hv0.w, hv0.z, hv0.y, hv0.x};
     int hs = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) hs += (int)hb[j];
     int htotal;
     const int hbefore = block_exclusive_scan(hs, sm.wa, htotal);
-    if (htotal == c) {  // (the same decision in every CTA: they read the same histogram)
+    if (htotal == c) {
       if (hbefore < n && hbefore + hs >= n) {
         int ab = hbefore;
 #pragma unroll
@@ -423,80 +446,128 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
         }
       }
       __syncthreads();
-      const uint32_t pb = (uint32_t)sm.pbin;
-      // this CTA's keys in the bin are listed (with their ids) in its own
-      // shared memory; its counts in and above the bin go to every CTA
-      int mine = 0, above_pb = 0;
-#pragma unroll U
-      for (int j = 0; j < KPT; ++j) {
-        const uint32_t top = keys.get(j) >> kPrefixShift;
-        const bool valid = first + j < c;
-        mine += valid && top == pb;
-        above_pb += valid && top > pb;
-      }
-      int cta2;  // one scan: candidates (low 16 bits), keys above the bin (high)
-      int pos = block_exclusive_scan(mine | (above_pb << 16), sm.wa, cta2) & 0xffff;
-      if (mine) {
-#pragma unroll U
-        for (int j = 0; j < KPT; ++j) {
-          const uint32_t k = keys.get(j);
-          if (first + j < c && (k >> kPrefixShift) == pb) {
-            if (pos < kSeg) sm.cand[pos] = make_uint2(k, (uint32_t)(first + j));
-            ++pos;
-          }
+      pb = (uint32_t)sm.pbin;
+      hist_ok = true;
+    }
+  }
+
+  // ---- keys into shared memory; on the histogram path, which of them lie
+  // above the bin (kept for sure) and in it (the candidates)
+  SmemKeys<KPT> keys{reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem)) + tid};
+  uint64_t above_mask = 0, cand_mask = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const bool valid = first + j < c;
+    const uint32_t k = valid ? order_key(sc[j]) : 0u;
+    keys.set(j, k);
+    if (valid && (k >> kPrefixShift) > pb) above_mask |= 1ull << j;
+    if (valid && (k >> kPrefixShift) == pb) cand_mask |= 1ull << j;
+  }
+
+  uint32_t prefix = 0;
+  int need = n;    // how many keys matching `prefix` are still to be taken
+  int mode = 0;    // how tau was found: 0 four cluster passes, 1 two passes and
+                   // the gathered candidates, 2 the prefix histogram
+  int ncand = 0;
+  bool hist_zeroed = false;
+
+  if (hist_ok) {
+    // this CTA's candidates are listed (with their ids) in its own shared
+    // memory; its counts in and above the bin go to every CTA
+    const int mine = __popcll((long long)cand_mask), above_pb = __popcll((long long)above_mask);
+    int cta2;  // one scan: candidates (low 16 bits), keys above the bin (high)
+    int pos = block_exclusive_scan(mine | (above_pb << 16), sm.wa, cta2) & 0xffff;
+    for (uint64_t m = cand_mask; m; m &= m - 1) {
+      const int j = __ffsll((long long)m) - 1;
+      if (pos < kSeg) sm.cand[pos] = make_uint2(keys.get(j), (uint32_t)(first + j));
+      ++pos;
+    }
+    if (tid < CL) {  // thread q tells CTA q
+      *cl.map_shared_rank(&sm.scnt[rank], tid) = cta2 & 0xffff;
+      *cl.map_shared_rank(&sm.sgt[rank], tid) = cta2 >> 16;
+    }
+    if (tid < kBins) {
+      sm.hw[0][tid] = 0u;
+      sm.hw[1][tid] = 0u;
+      sm.hw[2][tid] = 0u;
+    }
+    if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
+    if (tid == 0) sm.nfin = 0;
+    csync<CL>();  // lists and counts complete; every CTA has read the histogram
+    zero_hist_share<CL>(r.hrow, rank);
+    hist_zeroed = true;
+    // the histogram's bin is taken only when the exact counts confirm it
+    int in_bin = 0, above_bin = 0;
+    bool over = false;
+#pragma unroll
+    for (int q = 0; q < CL; ++q) {
+      in_bin += sm.scnt[q];
+      above_bin += sm.sgt[q];
+      over |= sm.scnt[q] > kSeg;
+    }
+    if (!over && above_bin < n && above_bin + in_bin >= n) {
+      mode = 2;
+      need = n - above_bin;
+      prefix = pb << kPrefixShift;
+      // ---- pull every CTA's list into registers (independent DSMEM loads):
+      // slot s of thread tid is entry (tid + s*kThreads) % kSeg of CTA
+      // (tid + s*kThreads) / kSeg; then release the lists for their CTAs' exit
+      uint2 ck[kSlots];
+      uint32_t valid = 0;
+#pragma unroll
+      for (int s = 0; s < kSlots; ++s) {
+        const int e = tid + s * kThreads, q = e / kSeg, i = e % kSeg;
+        ck[s] = make_uint2(0u, 0u);
+        if (i < sm.scnt[q]) {
+          ck[s] = *cl.map_shared_rank(&sm.cand[i], q);
+          valid |= 1u << s;
         }
       }
-      if (tid < CL) {  // thread q tells CTA q
-        *cl.map_shared_rank(&sm.scnt[rank], tid) = cta2 & 0xffff;
-        *cl.map_shared_rank(&sm.sgt[rank], tid) = cta2 >> 16;
-      }
-      if (tid < kBins) {
-        sm.hw[0][tid] = 0u;
-        sm.hw[1][tid] = 0u;
-        sm.hw[2][tid] = 0u;
-      }
-      if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
-      csync<CL>();  // lists and counts complete; every CTA has read the histogram
-      zero_hist_share<CL>(r.hrow, rank);
-      hist_zeroed = true;
-      // the histogram's bin is taken only when the exact counts confirm it
-      int in_bin = 0, above_bin = 0;
-      bool over = false;
+      asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+      // ---- key bits 12..19 over the candidates
 #pragma unroll
-      for (int q = 0; q < CL; ++q) {
-        in_bin += sm.scnt[q];
-        above_bin += sm.sgt[q];
-        over |= sm.scnt[q] > kSeg;
-      }
-      if (!over && above_bin < n && above_bin + in_bin >= n) {
-        mode = 2;
-        need = n - above_bin;
-        prefix = pb << kPrefixShift;
-        // ---- pull every CTA's list into registers (independent DSMEM loads):
-        // slot s of thread tid is entry (tid + s*kThreads) % kSeg of CTA
-        // (tid + s*kThreads) / kSeg; then release the lists for their CTAs' exit
-        uint32_t ck[kSlots];
-        uint32_t valid = 0;
+      for (int s = 0; s < kSlots; ++s)
+        if ((valid >> s) & 1u) atomicAdd(&sm.hw[0][(ck[s].x >> 12) & 255u], 1u);
+      __syncthreads();
+      if (tid < kBins)
+        find_bin((int)sm.hw[0][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[0], &sm.above[0], sm.wa);
+      __syncthreads();
+      prefix |= (uint32_t)sm.bin[0] << 12;
+      need -= sm.above[0];
+      const int m20 = (int)sm.hw[0][sm.bin[0]];  // candidates matching the 20-bit prefix
+      if (m20 <= kRankCap) {
+        // ---- those few, gathered, are ranked directly under (key desc, id
+        // asc): the one of rank need-1 is tau
 #pragma unroll
-        for (int s = 0; s < kSlots; ++s) {
-          const int e = tid + s * kThreads, q = e / kSeg, i = e % kSeg;
-          ck[s] = 0u;
-          if (i < sm.scnt[q]) {
-            ck[s] = cl.map_shared_rank(&sm.cand[i], q)->x;
-            valid |= 1u << s;
+        for (int s = 0; s < kSlots; ++s)
+          if (((valid >> s) & 1u) && (ck[s].x >> 12) == (prefix >> 12)) sm.fin[atomicAdd(&sm.nfin, 1)] = ck[s];
+        __syncthreads();
+        if (tid < m20) {
+          const uint2 me = sm.fin[tid];
+          int rk = 0, r_key = 0;  // rank, and candidates with a larger key
+          for (int i = 0; i < m20; ++i) {
+            const uint2 o = sm.fin[i];
+            rk += o.x > me.x || (o.x == me.x && o.y < me.y);
+            r_key += o.x > me.x;
+          }
+          if (rk == need - 1) {
+            sm.tau = me.x;
+            sm.above[2] = r_key;
           }
         }
-        asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-        // ---- the low 20 bits over the candidates: digits of 8, 8 and 4 bits
+        __syncthreads();
+        prefix = sm.tau;
+        need -= sm.above[2];
+      } else {
+        // ---- many ties in the bin: key bits 4..11, then 0..3
 #pragma unroll 1
-        for (int L = 0; L < 3; ++L) {
-          const int shift = L == 0 ? 12 : (L == 1 ? 4 : 0);
-          const int hi = L == 0 ? 20 : (L == 1 ? 12 : 4);  // key bits >= hi are fixed
+        for (int L = 1; L < 3; ++L) {
+          const int shift = L == 1 ? 4 : 0, hi = L == 1 ? 12 : 4;
           const uint32_t dmask = L == 2 ? 15u : 255u;
 #pragma unroll
           for (int s = 0; s < kSlots; ++s)
-            if (((valid >> s) & 1u) && (ck[s] >> hi) == (prefix >> hi))
-              atomicAdd(&sm.hw[L][(ck[s] >> shift) & dmask], 1u);
+            if (((valid >> s) & 1u) && (ck[s].x >> hi) == (prefix >> hi))
+              atomicAdd(&sm.hw[L][(ck[s].x >> shift) & dmask], 1u);
           __syncthreads();
           if (tid < kBins)
             find_bin((int)sm.hw[L][kBins - 1 - tid], need, kBins - 1 - tid, &sm.bin[L], &sm.above[L], sm.wa);
@@ -504,14 +575,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
           prefix |= (uint32_t)sm.bin[L] << shift;
           need -= sm.above[L];
         }
-        // per source CTA: candidates above and equal to tau
+      }
+      // per source CTA: candidates above and equal to tau
 #pragma unroll
-        for (int s = 0; s < kSlots; ++s) {
-          if ((valid >> s) & 1u) {
-            const int q = (tid + s * kThreads) / kSeg;
-            if (ck[s] > prefix) atomicAdd(&sm.ccnt[q], 1);
-            else if (ck[s] == prefix) atomicAdd(&sm.ccnt[kMaxCL + q], 1);
-          }
+      for (int s = 0; s < kSlots; ++s) {
+        if ((valid >> s) & 1u) {
+          const int q = (tid + s * kThreads) / kSeg;
+          if (ck[s].x > prefix) atomicAdd(&sm.ccnt[q], 1);
+          else if (ck[s].x == prefix) atomicAdd(&sm.ccnt[kMaxCL + q], 1);
         }
       }
     }
@@ -663,10 +734,24 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     }
   }
 
-  // ---- kept ids: all keys > tau, then the first `need` keys == tau by id
-  const int ge = count_vs<KPT>(keys, tau);
+  // ---- kept ids: all keys > tau, then the first `need` keys == tau by id.
+  // This thread's counts: on the histogram path from its masks (the keys
+  // above the bin, then its few candidates against tau), else from its keys.
+  int gt = 0, eq = 0;
+  if (mode == 2) {
+    gt = __popcll((long long)above_mask);
+    for (uint64_t m = cand_mask; m; m &= m - 1) {
+      const uint32_t k = keys.get(__ffsll((long long)m) - 1);
+      gt += k > tau;
+      eq += k == tau;
+    }
+  } else {
+    const int ge = count_vs<KPT>(keys, tau);
+    gt = ge & 0xffff;
+    eq = ge >> 16;
+  }
   int both;  // per-CTA counts stay below 2^16
-  const int before = block_exclusive_scan(ge, sm.wa, both);  // syncs: wsum, ccnt visible
+  const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);  // syncs: wsum, ccnt visible
   // the CTAs before this one: lane q of every warp takes CTA q's counts, and a
   // warp prefix over q gives the offsets (no serial loop, no extra barrier)
   int gt_q = 0, eq_q = 0;
@@ -698,8 +783,12 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
   const int eq_prev = __shfl_sync(0xffffffffu, eq_before_q, rank);
   int rem = need - eq_prev;  // tau-keys still to take at this CTA's start
   rem = rem < 0 ? 0 : rem;
-  emit_kept<KPT>(sm, keys, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff, both >> 16,
-                 rem, off, r, tvec);
+  if (mode == 2)
+    emit_kept<KPT, true>(sm, keys, above_mask, cand_mask, first, tau, gt, before & 0xffff, before >> 16,
+                         both & 0xffff, both >> 16, rem, off, r, tvec);
+  else
+    emit_kept<KPT, false>(sm, keys, 0, 0, first, tau, gt, before & 0xffff, before >> 16, both & 0xffff,
+                          both >> 16, rem, off, r, tvec);
   if (rank == 0) write_tail(a, r, t);
   // the other CTAs read this CTA's candidate list: stay until they have
   if (mode == 2) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
