@@ -358,26 +358,9 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
   }
   __syncthreads();
 
-  // ---- merge the warps.  Per head (one thread each): the max over the warps
-  // and every warp's rescale factor; then thread -> (head, 4 consecutive dims)
-  __shared__ float fac[NW][8];   // warp w's factor for head h
-  __shared__ float hml[8][2];    // the CTA's (max, sum) per head
-  if (tid < 8) {
-    const int h = tid;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, wml[w][h][0]);
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const float mw = wml[w][h][0];
-      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);  // -inf: the warp had no tokens
-      fac[w][h] = f;
-      L = fmaf(wml[w][h][1], f, L);
-    }
-    hml[h][0] = M;
-    hml[h][1] = L;
-  }
+  // ---- merge the warps.  Every thread merges its items (head h, dims d..d+3)
+  // itself: the head's max over the warps and each warp's rescale factor come
+  // from the warps' (max, sum), so no per-head pass and no extra barrier.
   // The cluster's outputs are split among its CTAs: CTA r finishes items
   // [r * PER, (r + 1) * PER).  Every CTA pushes its share of item i (and its
   // per-head max and sum) into the owner's receive slots before ONE cluster
@@ -386,69 +369,61 @@ __global__ void __launch_bounds__(kClWarps * 32, 1)
   constexpr int PER = (ITEMS8 + CL - 1) / CL;
   __shared__ float4 recv_o[CL][PER];
   __shared__ float recv_ml[CL][8][2];
-  __syncthreads();
   const size_t th0 = (size_t)t * a.Hq + h0;
   const int items = G * (D / 4);
-  if constexpr (CL > 1) {
-    if (tid < 8 * CL) {
-      const int q = tid / 8, h = tid % 8;
-      float* dst = cl.map_shared_rank(&recv_ml[0][0][0], q);
-      dst[(rank * 8 + h) * 2] = hml[h][0];
-      dst[(rank * 8 + h) * 2 + 1] = hml[h][1];
-    }
-  }
   for (int idx = tid; idx < items; idx += NT) {
     const int h = idx / (D / 4), d = 4 * (idx % (D / 4));
     // every slot is written (zeros for warps without tiles): all loads go out at once
     float4 v[NW];
 #pragma unroll
     for (int w = 0; w < NW; ++w) v[w] = ld_o4<SH>(wo_dyn + (w * 8 + h) * OS, d);
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, wml[w][h][0]);
+    float L = 0.f;
     float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float f = fac[w][h];
+      const float mw = wml[w][h][0];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);  // -inf: the warp had no tokens
+      L = fmaf(wml[w][h][1], f, L);
       O.x = fmaf(v[w].x, f, O.x); O.y = fmaf(v[w].y, f, O.y); O.z = fmaf(v[w].z, f, O.z); O.w = fmaf(v[w].w, f, O.w);
     }
     if constexpr (CL == 1) {
-      write_out<OT, D>(a, th0 + h, d, O, hml[h][0], hml[h][1], vmul);
+      write_out<OT, D>(a, th0 + h, d, O, M, L, vmul);
     } else {
       const int owner = idx / PER;
       *cl.map_shared_rank(&recv_o[rank][idx - owner * PER], owner) = O;
+      if (d == 0) {  // the CTA's (max, sum) of head h, to every CTA
+#pragma unroll
+        for (int q = 0; q < CL; ++q) {
+          float* dst = cl.map_shared_rank(&recv_ml[rank][h][0], q);
+          dst[0] = M;
+          dst[1] = L;
+        }
+      }
     }
   }
   if constexpr (CL > 1) {
     cl.sync();  // every push has landed; from here every access is local
-    __shared__ float cfac[CL][8];
-    __shared__ float cml[8][2];
-    if (tid < 8) {
-      const int h = tid;
-      float M = -INFINITY;
-#pragma unroll
-      for (int q = 0; q < CL; ++q) M = fmaxf(M, recv_ml[q][h][0]);
-      float L = 0.f;
-#pragma unroll
-      for (int q = 0; q < CL; ++q) {
-        const float mq = recv_ml[q][h][0];
-        const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
-        cfac[q][h] = f;
-        L = fmaf(recv_ml[q][h][1], f, L);
-      }
-      cml[h][0] = M;
-      cml[h][1] = L;
-    }
-    __syncthreads();
     const int lo = rank * PER;
     const int hi = lo + PER < items ? lo + PER : items;
     for (int idx = lo + tid; idx < hi; idx += NT) {
       const int h = idx / (D / 4), d = 4 * (idx % (D / 4));
+      float M = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < CL; ++q) M = fmaxf(M, recv_ml[q][h][0]);
+      float L = 0.f;
       float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int q = 0; q < CL; ++q) {
-        const float f = cfac[q][h];
+        const float mq = recv_ml[q][h][0];
+        const float f = mq == -INFINITY ? 0.f : exp2f(mq - M);
+        L = fmaf(recv_ml[q][h][1], f, L);
         const float4 v = recv_o[q][idx - lo];
         O.x = fmaf(v.x, f, O.x); O.y = fmaf(v.y, f, O.y); O.z = fmaf(v.z, f, O.z); O.w = fmaf(v.w, f, O.w);
       }
-      write_out<OT, D>(a, th0 + h, d, O, cml[h][0], cml[h][1], vmul);
+      write_out<OT, D>(a, th0 + h, d, O, M, L, vmul);
     }
   }
 }
