@@ -278,45 +278,65 @@ def pack_inputs(st):
 def time_e2e(sets, steps, warmup, stream):
     """Through the public API with host buffers: every step copies its
     query-side inputs from pinned host memory to the device (one packed
-    copy), runs the calls and copies the output back to pinned host memory;
-    the steps are captured once as CUDA graphs (one per input set) and
-    replayed.  The KV cache and the indexer keys are resident device state."""
+    copy), runs the calls and copies the output back to pinned host memory.
+    The copies run on two copy streams, so step i+1's inputs go up and step
+    i's output comes down while the kernels of step i (i+1) run; events keep
+    each buffer safe (a set's inputs are overwritten only after the kernels
+    that read them, its output only after its previous copy-out).  The K
+    timed steps are one captured CUDA graph.  The KV cache and the indexer
+    keys are resident device state."""
     hosts = []
     for st in sets:
         dev, host = pack_inputs(st)
         hosts.append((host, dev, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()))
     h2d = hosts[0][1].numel()
     d2h = hosts[0][2].numel() * hosts[0][2].element_size()
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(sets)
 
-    def one(i):
-        st = sets[i % len(sets)]
-        hin, dev_in, hout = hosts[i % len(sets)]
-        dev_in.copy_(hin, non_blocking=True)
-        st.run()
-        hout.copy_(st.out, non_blocking=True)
+    def steps_on(main, count):
+        ev_h = [torch.cuda.Event() for _ in range(count)]
+        ev_k = [torch.cuda.Event() for _ in range(count)]
+        ev_d = [torch.cuda.Event() for _ in range(count)]
+        cin.wait_stream(main)
+        cout.wait_stream(main)
+        for i in range(count):
+            st = sets[i % n]
+            hin, dev_in, hout = hosts[i % n]
+            with torch.cuda.stream(cin):
+                if i >= n:
+                    cin.wait_event(ev_k[i - n])   # the kernels that read this set's inputs are done
+                dev_in.copy_(hin, non_blocking=True)
+                ev_h[i].record(cin)
+            main.wait_event(ev_h[i])
+            if i >= n:
+                main.wait_event(ev_d[i - n])      # this set's previous output has been copied out
+            st.run(main)
+            ev_k[i].record(main)
+            with torch.cuda.stream(cout):
+                cout.wait_event(ev_k[i])
+                hout.copy_(st.out, non_blocking=True)
+                ev_d[i].record(cout)
+        main.wait_stream(cin)
+        main.wait_stream(cout)
 
     with torch.cuda.stream(stream):
-        for i in range(warmup):
-            one(i)
+        steps_on(stream, warmup)
         torch.cuda.synchronize()
-        graphs = []
-        for i in range(len(sets)):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g):
-                one(i)
-            graphs.append(g)
-        for g in graphs:
-            g.replay()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            steps_on(stream, steps)
+        g.replay()
         torch.cuda.synchronize()
         barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        g.replay()
         b.record()
     torch.cuda.synchronize()
     barrier()
+    del g
     return a.elapsed_time(b), h2d, d2h
 
 
