@@ -13,8 +13,9 @@
 //  * the warp streams its row's 16-token tiles through a private ring of S
 //    shared-memory stages with 16-byte cp.async (no registers held while in
 //    flight; S - 1 tiles in flight while one is computed).  The 16-byte chunk
-//    c of staged row r sits at chunk position c ^ (r & 7), which makes the
-//    fragment reads below bank-conflict-free;
+//    c of staged row r sits at chunk position c ^ sw(r), sw(r) = (r & 7) ^
+//    4 (r & 1): the K reads (rows g, g+1 in a quarter-warp) and the V reads
+//    (rows 2tq) then fall on distinct banks;
 //  * per tile: S^T = K.Q^T on m16n8k16 (tokens as M, heads as N; the K
 //    fragments serve both head tiles), an online softmax per head in base 2,
 //    and O^T += V^T.P^T with V rows paired by byte permutes;
@@ -42,6 +43,9 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait_pf() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
+
+// swizzle of the 16-byte chunks of staged row r (see the file comment)
+__device__ __forceinline__ int pf_sw(int r) { return (r & 7) ^ ((r & 1) << 2); }
 
 template <bool FP8, int D>
 constexpr int pf_stages() {
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
       for (int rr0 = 0; rr0 < 16; rr0 += RPP) {
         const int rr = rr0 + lane / NCH;
         const long long o = __shfl_sync(0xffffffffu, off, rr);
-        const uint32_t pos = (uint32_t)(((c ^ (rr & 7)) * 16));
+        const uint32_t pos = (uint32_t)(((c ^ pf_sw(rr)) * 16));
         const uint32_t dk = sb + rr * ROWB + pos, dv = sb + (16 + rr) * ROWB + pos;
         if (o >= 0) {
           cp_async16_pf(dk, kbase + o + c * 16);
@@ -163,13 +167,13 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
     const unsigned vmask = valid_s[warp][i % S];
     const bool ok0 = (vmask >> g) & 1u, ok1 = (vmask >> (g + 8)) & 1u;
 
-    // ---- S^T = K . Q^T for every head tile (rows g, g+8 have row & 7 == g)
+    // ---- S^T = K . Q^T for every head tile (rows g and g+8 share a swizzle)
     float sc[NT][4];
 #pragma unroll
     for (int u = 0; u < NT; ++u) sc[u][0] = sc[u][1] = sc[u][2] = sc[u][3] = 0.f;
 #pragma unroll
     for (int j = 0; j < KJ; ++j) {
-      const int pc = ((4 * j + tq) ^ g) * 16;
+      const int pc = ((4 * j + tq) ^ pf_sw(g)) * 16;
       const uint4 k0 = lds16(ks + g * ROWB + pc);
       const uint4 k1 = lds16(ks + (g + 8) * ROWB + pc);
       const uint32_t w0[4] = {k0.x, k0.y, k0.z, k0.w};
@@ -233,15 +237,16 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
       pb[u][1] = movmatrix_trans(pack2<FP8>(p2, p3));  // tokens 8..15
     }
 
-    // ---- O^T += V^T . P^T; staged V rows 2tq, 2tq+1, 2tq+8, 2tq+9 have
-    // row & 7 == 2tq, 2tq+1, 2tq, 2tq+1.  The V fragments serve every head tile.
+    // ---- O^T += V^T . P^T; staged V rows 2tq, 2tq+1, 2tq+8, 2tq+9 have the
+    // swizzles of rows 2tq, 2tq+1, 2tq, 2tq+1.  The V fragments serve every head tile.
 #pragma unroll
     for (int j = 0; j < VJ; ++j) {
       const int c = g + 8 * j;
-      const uint4 A = lds16(vs + (2 * tq) * ROWB + ((c ^ (2 * tq)) * 16));
-      const uint4 B = lds16(vs + (2 * tq + 1) * ROWB + ((c ^ (2 * tq + 1)) * 16));
-      const uint4 C = lds16(vs + (2 * tq + 8) * ROWB + ((c ^ (2 * tq)) * 16));
-      const uint4 E = lds16(vs + (2 * tq + 9) * ROWB + ((c ^ (2 * tq + 1)) * 16));
+      const int sa = pf_sw(2 * tq), sb = pf_sw(2 * tq + 1);
+      const uint4 A = lds16(vs + (2 * tq) * ROWB + ((c ^ sa) * 16));
+      const uint4 B = lds16(vs + (2 * tq + 1) * ROWB + ((c ^ sb) * 16));
+      const uint4 C = lds16(vs + (2 * tq + 8) * ROWB + ((c ^ sa) * 16));
+      const uint4 E = lds16(vs + (2 * tq + 9) * ROWB + ((c ^ sb) * 16));
       const uint32_t va[4] = {A.x, A.y, A.z, A.w};  // token 2tq
       const uint32_t vb[4] = {B.x, B.y, B.z, B.w};  // token 2tq+1
       const uint32_t vc[4] = {C.x, C.y, C.z, C.w};  // token 2tq+8
