@@ -402,13 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
   }
   const int c = r.c, n = r.n;
 
-  // ---- loads: the prefix histogram (8 bins per thread, from the top) and
-  // this thread's KPT consecutive scores
-  uint4 hv0 = make_uint4(0u, 0u, 0u, 0u), hv1 = hv0;
-  if (r.hrow) {
-    hv0 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 8 - 8 * tid));
-    hv1 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 4 - 8 * tid));
-  }
+  // ---- loads: this thread's KPT consecutive scores, then the prefix
+  // histogram (8 bins per thread, from the top)
   const int first = (rank * kThreads + tid) * KPT;
   const float* row = a.scores + (size_t)t * a.score_stride;
   float sc[KPT];
@@ -424,6 +419,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc[j + e] = first + j + e < c ? __ldg(row + first + j + e) : 0.f;
     }
+  }
+  uint4 hv0 = make_uint4(0u, 0u, 0u, 0u), hv1 = hv0;
+  if (r.hrow) {
+    hv0 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 8 - 8 * tid));
+    hv1 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 4 - 8 * tid));
   }
 
   // ---- the bin of the n-th largest key, from the histogram
@@ -469,7 +469,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
   int mode = 0;    // how tau was found: 0 four cluster passes, 1 two passes and
                    // the gathered candidates, 2 the prefix histogram
   int ncand = 0;
-  bool hist_zeroed = false;
 
   if (hist_ok) {
     // this CTA's candidates are listed (with their ids) in its own shared
@@ -494,8 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     if (tid < 2 * kMaxCL) sm.ccnt[tid] = 0;
     if (tid == 0) sm.nfin = 0;
     csync<CL>();  // lists and counts complete; every CTA has read the histogram
-    zero_hist_share<CL>(r.hrow, rank);
-    hist_zeroed = true;
+    // (the histogram is zeroed below while the DSMEM pulls are in flight, or in cluster pass 0)
     // the histogram's bin is taken only when the exact counts confirm it
     int in_bin = 0, above_bin = 0;
     bool over = false;
@@ -523,6 +521,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
           valid |= 1u << s;
         }
       }
+      zero_hist_share<CL>(r.hrow, rank);
       asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
       // ---- key bits 12..19 over the candidates
 #pragma unroll
@@ -614,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
         for (int q = 0; q < CL; ++q) cl.map_shared_rank(&sm.hall[pass][rank][tid], q)[0] = v;
       }
       csync<CL>();  // every CTA's counts are in every CTA's table
-      if (pass == 0 && r.hrow && !hist_zeroed) zero_hist_share<CL>(r.hrow, rank);
+      if (pass == 0 && r.hrow && mode != 2) zero_hist_share<CL>(r.hrow, rank);
       if (tid < kBins) {
         int h = 0;
 #pragma unroll
