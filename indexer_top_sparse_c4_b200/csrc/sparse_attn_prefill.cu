@@ -7,23 +7,27 @@
 // gathered for it alone: 1 KiB per token and KV head at D = 256 BF16, about
 // 34 GB for an 8,192-query chunk, served mostly from L2.  The kernel is built
 // to move those bytes once and keep many of them in flight:
-//  * one warp per (query, KV head) row handles ALL query heads of the KV head
-//    (up to 16, as two n8 MMA tiles), so each K/V row is gathered once per
-//    row, not once per group of 8 heads;
-//  * the warp streams its row's 16-token tiles through a private ring of S
-//    shared-memory stages with 16-byte cp.async (no registers held while in
-//    flight; S - 1 tiles in flight while one is computed).  The 16-byte chunk
+//  * each (query, KV head) row gathers every K/V row once for ALL query
+//    heads of the KV head: one warp per n8 tile of heads (two warps for 9-16
+//    heads), sharing the row's staged tiles.  Two warps of ~130 registers
+//    instead of one of 255 double the warps an SM holds to hide latency;
+//  * the row's warps stream its 16-token tiles through a ring of S
+//    shared-memory stages with 16-byte cp.async (each warp copies its share
+//    of the rows; no registers held while in flight; S - 1 tiles in flight
+//    while one is computed), meeting at one named barrier per tile.  The 16-byte chunk
 //    c of staged row r sits at chunk position c ^ sw(r), sw(r) = (r & 7) ^
 //    4 (r & 1): the K reads (rows g, g+1 in a quarter-warp) and the V reads
 //    (rows 2tq) then fall on distinct banks;
-//  * per tile: S^T = K.Q^T on m16n8k16 (tokens as M, heads as N; the K
-//    fragments serve both head tiles), an online softmax per head in base 2,
-//    and O^T += V^T.P^T with V rows paired by byte permutes;
+//  * per tile: S^T = K.Q^T on m16n8k16 (tokens as M, heads as N), an
+//    online softmax per head in base 2, and O^T += V^T.P^T with V rows
+//    paired by byte permutes;
 //  * rows run KV head by KV head, so the cache lines being gathered at any
 //    time belong to one KV head: half the cache (64 MB for the 65,536-token
 //    BF16 chunk), which stays in L2 while every query of the chunk reads it;
-//  * the row's output is written by the warp itself: no merge, no workspace.
+//  * each warp writes its heads of the row's output: no merge, no workspace.
 #include <math.h>
+
+#include <type_traits>
 
 #include "attn_common.cuh"
 
@@ -32,7 +36,12 @@ namespace {
 
 using namespace attn;
 
-constexpr int kPfWarps = 7;                 // warps (rows) per CTA
+// (query, KV head) rows per CTA: 7 rows of one warp, or 6 rows of two warps
+// (12 warps of up to 168 registers; 14 would cap them at 128 and spill)
+template <int NT>
+constexpr int pf_rows() {
+  return NT > 1 ? 6 : 7;
+}
 constexpr int kPfRingBytes = 224 * 1024;    // per CTA
 
 __device__ __forceinline__ void cp_async16_pf(uint32_t smem_addr, const void* gptr) {
@@ -47,34 +56,38 @@ __device__ __forceinline__ void cp_async_wait_pf() {
 // swizzle of the 16-byte chunks of staged row r (see the file comment)
 __device__ __forceinline__ int pf_sw(int r) { return (r & 7) ^ ((r & 1) << 2); }
 
-template <bool FP8, int D>
+template <bool FP8, int D, int NT>
 constexpr int pf_stages() {
   constexpr int stage = 32 * Geo<FP8, D>::ROWB;  // 16 K rows + 16 V rows
-  constexpr int s = kPfRingBytes / kPfWarps / stage;
+  constexpr int s = kPfRingBytes / pf_rows<NT>() / stage;
   return s > 8 ? 8 : s;
 }
 
-// grid: ceil(T * Hkv / kPfWarps) CTAs; warp w of CTA b takes row
-// b * kPfWarps + w = kvh * T + t (query t, KV head kvh).  NT n8 tiles cover
-// the G query heads of the KV head.
+// grid: ceil(T * Hkv / R) CTAs of R = pf_rows<NT>() row slots.  The NT warps of
+// slot j of CTA b take row b * R + j = kvh * T + t (query t, KV head
+// kvh); warp u of a row computes head tile u (heads 8u .. 8u+7 of the G of
+// the KV head) and stages tokens 16/NT * u .. of every tile.
 template <bool FP8, int D, typename QT, typename OT, int NT>
-__global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs a, float qk_scale, float vmul,
-                                                                       int rows) {
+__global__ void __launch_bounds__(pf_rows<NT>() * NT * 32, 1) attn_prefill_kernel(AttnArgs a, float qk_scale, float vmul,
+                                                                           int rows) {
   using G_ = Geo<FP8, D>;
   constexpr int CH = G_::CH, NCH = G_::NCH, KJ = G_::KJ, KS = G_::KS, NKS = G_::NKS, VJ = G_::VJ, MT = G_::MT,
                 MTJ = G_::MTJ, ROWB = G_::ROWB;
-  constexpr int S = pf_stages<FP8, D>();
+  constexpr int R = pf_rows<NT>();
+  constexpr int S = pf_stages<FP8, D, NT>();
   constexpr int STAGE = 32 * ROWB;
   static_assert(S >= 2, "at least two stages");
-  constexpr int RPP = 32 / NCH;  // rows a lane pass covers when staging
-  static_assert(NCH >= 8 && 32 % NCH == 0, "row chunks must swizzle over 8 and tile a warp");
+  constexpr int TPW = 16 / NT;    // token rows of a tile each warp of the row stages
+  constexpr int RPP = 32 / NCH;   // rows a lane pass covers when staging
+  static_assert(NCH >= 8 && 32 % NCH == 0 && TPW % RPP == 0, "row chunks must swizzle over 8 and tile a warp");
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint32_t valid_s[kPfWarps][8];  // per stage: bit i = token slot i of the tile is real
+  __shared__ uint32_t valid_s[R][8][NT];  // per stage and warp: bit i = token slot i of the tile is real
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int slot = warp / NT, u = warp % NT;
   const int g = lane >> 2, tq = lane & 3;
-  const int row = blockIdx.x * kPfWarps + warp;
+  const int row = blockIdx.x * R + slot;
   pdl_wait();
-  if (row >= rows) return;
+  if (row >= rows) return;  // (every warp of the row)
   // KV-head-major order: while the first half of the grid runs, only KV head
   // 0's cache lines are gathered (half the cache, which fits in L2)
   const int kvh = row / a.T, t = row % a.T;
@@ -85,7 +98,7 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
   int nt = a.n_tok[t];
   nt = nt < 0 ? 0 : (nt > a.W ? a.W : nt);
   if (r < 0 || r >= a.pt_rows) {
-    if (lane == 0 && kvh == 0) flag(a.status, QSA_DEV_BAD_REQUEST);
+    if (lane == 0 && kvh == 0 && u == 0) flag(a.status, QSA_DEV_BAD_REQUEST);
     r = 0;
     nt = 0;
   }
@@ -94,24 +107,32 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
   const size_t row_bytes = (size_t)a.Hkv * ROWB;
   const unsigned char* kbase = reinterpret_cast<const unsigned char*>(a.k_pages);
   const unsigned char* vbase = reinterpret_cast<const unsigned char*>(a.v_pages);
-  unsigned char* ring = smem + (size_t)warp * S * STAGE;
+  unsigned char* ring = smem + (size_t)slot * S * STAGE;
   const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
   const int ntiles = (nt + 15) / 16;
+  // the row's warps meet once per tile: every warp's copies of the tile have
+  // landed, and every warp is done with the stage the next copies refill
+  auto row_sync = [&]() {
+    if constexpr (NT > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(NT * 32) : "memory");
+    else __syncwarp();
+  };
 
-  // stage tile i (slots 16i .. 16i+15): lanes 0..15 look the rows up, then
-  // lane l copies chunk l % NCH of rows l / NCH, l / NCH + RPP, ... of K and V
-  // (a warp instruction moves whole 512-byte stretches of a row)
+  // stage this warp's TPW token rows of tile i: lanes 0..TPW-1 look the rows
+  // up, then lane l copies chunk l % NCH of rows l / NCH, l / NCH + RPP, ...
+  // of K and V (a warp instruction moves whole 512-byte stretches of a row)
   auto issue = [&](int i) {
     if (i < ntiles) {
-      const long long off = lane < 16 ? row_offset(a, trow, pt, 16 * i + lane, nt, kvh, row_bytes, ROWB) : -1;
-      const unsigned vmask = __ballot_sync(0xffffffffu, off >= 0) & 0xffffu;
-      if (lane == 0) valid_s[warp][i % S] = vmask;
+      const long long off =
+          lane < TPW ? row_offset(a, trow, pt, 16 * i + TPW * u + lane, nt, kvh, row_bytes, ROWB) : -1;
+      const unsigned vm = __ballot_sync(0xffffffffu, off >= 0) & ((1u << TPW) - 1u);
+      if (lane == 0) valid_s[slot][i % S][u] = vm << (TPW * u);
       const uint32_t sb = ring_s + (uint32_t)((i % S) * STAGE);
       const int c = lane % NCH;
 #pragma unroll
-      for (int rr0 = 0; rr0 < 16; rr0 += RPP) {
-        const int rr = rr0 + lane / NCH;
-        const long long o = __shfl_sync(0xffffffffu, off, rr);
+      for (int r0 = 0; r0 < TPW; r0 += RPP) {
+        const int lr = r0 + lane / NCH;  // row within this warp's share
+        const int rr = TPW * u + lr;     // row within the tile
+        const long long o = __shfl_sync(0xffffffffu, off, lr);
         const uint32_t pos = (uint32_t)(((c ^ pf_sw(rr)) * 16));
         const uint32_t dk = sb + rr * ROWB + pos, dv = sb + (16 + rr) * ROWB + pos;
         if (o >= 0) {
@@ -129,48 +150,40 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
   for (int i = 0; i < S - 1; ++i) issue(i);
 
   // Q^T B fragments of heads h0 + 8u + g (zero past G), head dim permuted like K
-  uint32_t qb[NT][NKS][2];
+  uint32_t qb[NKS][2];
   {
+    const int hg = 8 * u + g;
+    const QT* qrow = reinterpret_cast<const QT*>(a.q) + ((size_t)t * a.Hq + h0 + (hg < G ? hg : 0)) * D;
 #pragma unroll
-    for (int u = 0; u < NT; ++u) {
-      const int hg = 8 * u + g;
-      const QT* qrow = reinterpret_cast<const QT*>(a.q) + ((size_t)t * a.Hq + h0 + (hg < G ? hg : 0)) * D;
+    for (int j = 0; j < KJ; ++j) {
 #pragma unroll
-      for (int j = 0; j < KJ; ++j) {
+      for (int q4 = 0; q4 < KS; ++q4) {
+        const int d0 = CH * (4 * j + tq) + 4 * q4;
+        float v[4];
 #pragma unroll
-        for (int q4 = 0; q4 < KS; ++q4) {
-          const int d0 = CH * (4 * j + tq) + 4 * q4;
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[e] = hg < G ? Elem<QT>::get(qrow, d0 + e) : 0.f;
-          qb[u][j * KS + q4][0] = pack2<FP8>(v[0], v[1]);
-          qb[u][j * KS + q4][1] = pack2<FP8>(v[2], v[3]);
-        }
+        for (int e = 0; e < 4; ++e) v[e] = hg < G ? Elem<QT>::get(qrow, d0 + e) : 0.f;
+        qb[j * KS + q4][0] = pack2<FP8>(v[0], v[1]);
+        qb[j * KS + q4][1] = pack2<FP8>(v[2], v[3]);
       }
     }
   }
-  float m[NT][2], l[NT][2], o[NT][MT][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, o[MT][4];
 #pragma unroll
-  for (int u = 0; u < NT; ++u) {
-    m[u][0] = m[u][1] = -INFINITY;
-    l[u][0] = l[u][1] = 0.f;
-#pragma unroll
-    for (int i = 0; i < MT; ++i) o[u][i][0] = o[u][i][1] = o[u][i][2] = o[u][i][3] = 0.f;
-  }
+  for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
 
   for (int i = 0; i < ntiles; ++i) {
+    cp_async_wait_pf<S - 2>();      // this warp's copies of tile i have landed
+    row_sync();                     // ... and every warp's; all are done with tile i - 1
     issue(i + S - 1);               // into the stage tile i - 1 used
-    cp_async_wait_pf<S - 1>();      // this lane's copies of tile i have landed
-    __syncwarp();                   // ... and every lane's
     const unsigned char* ks = ring + (size_t)(i % S) * STAGE;
     const unsigned char* vs = ks + 16 * ROWB;
-    const unsigned vmask = valid_s[warp][i % S];
+    unsigned vmask = 0;
+#pragma unroll
+    for (int w = 0; w < NT; ++w) vmask |= valid_s[slot][i % S][w];
     const bool ok0 = (vmask >> g) & 1u, ok1 = (vmask >> (g + 8)) & 1u;
 
-    // ---- S^T = K . Q^T for every head tile (rows g and g+8 share a swizzle)
-    float sc[NT][4];
-#pragma unroll
-    for (int u = 0; u < NT; ++u) sc[u][0] = sc[u][1] = sc[u][2] = sc[u][3] = 0.f;
+    // ---- S^T = K . Q^T for this warp's head tile (rows g and g+8 share a swizzle)
+    float sc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < KJ; ++j) {
       const int pc = ((4 * j + tq) ^ pf_sw(g)) * 16;
@@ -187,27 +200,24 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
           af[1] = e4m3x2_to_f16x2(w1[q4]);
           af[2] = e4m3x2_to_f16x2(w0[q4] >> 16);
           af[3] = e4m3x2_to_f16x2(w1[q4] >> 16);
-#pragma unroll
-          for (int u = 0; u < NT; ++u) mma_f16(sc[u], af, qb[u][kk][0], qb[u][kk][1]);
+          mma_f16(sc, af, qb[kk][0], qb[kk][1]);
         } else {              // two words = 4 bf16 = dims 4q4..4q4+3 of the chunk
           af[0] = w0[2 * q4];
           af[1] = w1[2 * q4];
           af[2] = w0[2 * q4 + 1];
           af[3] = w1[2 * q4 + 1];
-#pragma unroll
-          for (int u = 0; u < NT; ++u) mma_bf16(sc[u], af, qb[u][kk][0], qb[u][kk][1]);
+          mma_bf16(sc, af, qb[kk][0], qb[kk][1]);
         }
       }
     }
 
-    // ---- online softmax per head tile, heads 8u + 2tq (s0, s2) and 8u + 2tq + 1 (s1, s3)
-    uint32_t pb[NT][2];
-#pragma unroll
-    for (int u = 0; u < NT; ++u) {
-      const float s0 = ok0 ? sc[u][0] * qk_scale : -INFINITY;
-      const float s1 = ok0 ? sc[u][1] * qk_scale : -INFINITY;
-      const float s2 = ok1 ? sc[u][2] * qk_scale : -INFINITY;
-      const float s3 = ok1 ? sc[u][3] * qk_scale : -INFINITY;
+    // ---- online softmax, heads 8u + 2tq (s0, s2) and 8u + 2tq + 1 (s1, s3)
+    uint32_t pb[2];
+    {
+      const float s0 = ok0 ? sc[0] * qk_scale : -INFINITY;
+      const float s1 = ok0 ? sc[1] * qk_scale : -INFINITY;
+      const float s2 = ok1 ? sc[2] * qk_scale : -INFINITY;
+      const float s3 = ok1 ? sc[3] * qk_scale : -INFINITY;
       float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
 #pragma unroll
       for (int d = 4; d <= 16; d <<= 1) {
@@ -217,28 +227,28 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
       // the base moves only when the max grows by more than 8 (log2 units): p
       // stays below 2^8 and the FP32 sums keep their accuracy, while most tiles
       // skip the rescale of the accumulators
-      const float mn0 = mx0 > m[u][0] + 8.f ? mx0 : m[u][0];
-      const float mn1 = mx1 > m[u][1] + 8.f ? mx1 : m[u][1];
+      const float mn0 = mx0 > m0 + 8.f ? mx0 : m0;
+      const float mn1 = mx1 > m1 + 8.f ? mx1 : m1;
       const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = m[u][0] == -INFINITY ? 0.f : exp2f(m[u][0] - b0);
-      const float al1 = m[u][1] == -INFINITY ? 0.f : exp2f(m[u][1] - b1);
+      const float al0 = m0 == -INFINITY ? 0.f : exp2f(m0 - b0);
+      const float al1 = m1 == -INFINITY ? 0.f : exp2f(m1 - b1);
       const float p0 = exp2f(s0 - b0), p1 = exp2f(s1 - b1), p2 = exp2f(s2 - b0), p3 = exp2f(s3 - b1);
-      m[u][0] = mn0;
-      m[u][1] = mn1;
-      l[u][0] = l[u][0] * al0 + p0 + p2;
-      l[u][1] = l[u][1] * al1 + p1 + p3;
+      m0 = mn0;
+      m1 = mn1;
+      l0 = l0 * al0 + p0 + p2;
+      l1 = l1 * al1 + p1 + p3;
       if (!__all_sync(0xffffffffu, al0 == 1.f && al1 == 1.f)) {
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          o[u][mt][0] *= al0; o[u][mt][1] *= al1; o[u][mt][2] *= al0; o[u][mt][3] *= al1;
+          o[mt][0] *= al0; o[mt][1] *= al1; o[mt][2] *= al0; o[mt][3] *= al1;
         }
       }
-      pb[u][0] = movmatrix_trans(pack2<FP8>(p0, p1));  // tokens 0..7
-      pb[u][1] = movmatrix_trans(pack2<FP8>(p2, p3));  // tokens 8..15
+      pb[0] = movmatrix_trans(pack2<FP8>(p0, p1));  // tokens 0..7
+      pb[1] = movmatrix_trans(pack2<FP8>(p2, p3));  // tokens 8..15
     }
 
     // ---- O^T += V^T . P^T; staged V rows 2tq, 2tq+1, 2tq+8, 2tq+9 have the
-    // swizzles of rows 2tq, 2tq+1, 2tq, 2tq+1.  The V fragments serve every head tile.
+    // swizzles of rows 2tq, 2tq+1, 2tq, 2tq+1
 #pragma unroll
     for (int j = 0; j < VJ; ++j) {
       const int c = g + 8 * j;
@@ -268,11 +278,8 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
           ag[1] = e4m3x2_to_f16x2(hi01 >> 16);
           ag[2] = e4m3x2_to_f16x2(hi89);
           ag[3] = e4m3x2_to_f16x2(hi89 >> 16);
-#pragma unroll
-          for (int u = 0; u < NT; ++u) {
-            mma_f16(o[u][mt], af, pb[u][0], pb[u][1]);
-            mma_f16(o[u][mt + 1], ag, pb[u][0], pb[u][1]);
-          }
+          mma_f16(o[mt], af, pb[0], pb[1]);
+          mma_f16(o[mt + 1], ag, pb[0], pb[1]);
         } else {
           const int mt = j * MTJ + wd;
           uint32_t af[4];
@@ -280,47 +287,41 @@ __global__ void __launch_bounds__(kPfWarps * 32, 1) attn_prefill_kernel(AttnArgs
           af[1] = __byte_perm(va[wd], vb[wd], 0x7632);
           af[2] = __byte_perm(vc[wd], vd[wd], 0x5410);
           af[3] = __byte_perm(vc[wd], vd[wd], 0x7632);
-#pragma unroll
-          for (int u = 0; u < NT; ++u) mma_bf16(o[u][mt], af, pb[u][0], pb[u][1]);
+          mma_bf16(o[mt], af, pb[0], pb[1]);
         }
       }
     }
-    __syncwarp();  // every lane is done with the stage before it is refilled
   }
   cp_async_wait_pf<0>();
   pdl_launch_dependents();
 
-  // ---- the row's output: heads 8u + 2tq (c0, c2) and 8u + 2tq + 1 (c1, c3);
-  // rows g / g+8 of m-tile mt are dims d_lo / d_lo + 1
+  // ---- this warp's heads of the row's output: heads 8u + 2tq (c0, c2) and
+  // 8u + 2tq + 1 (c1, c3); rows g / g+8 of m-tile mt are dims d_lo / d_lo + 1
   const size_t th0 = (size_t)t * a.Hq + h0;
 #pragma unroll
-  for (int u = 0; u < NT; ++u) {
-    float l0 = l[u][0], l1 = l[u][1];
+  for (int d = 4; d <= 16; d <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, d);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, d);
+  }
+  const float inv0 = l0 > 0.f ? vmul / l0 : 0.f, inv1 = l1 > 0.f ? vmul / l1 : 0.f;
+  const int ha = 8 * u + 2 * tq, hb = ha + 1;
 #pragma unroll
-    for (int d = 4; d <= 16; d <<= 1) {
-      l0 += __shfl_xor_sync(0xffffffffu, l0, d);
-      l1 += __shfl_xor_sync(0xffffffffu, l1, d);
+  for (int mt = 0; mt < MT; ++mt) {
+    const int d_lo = CH * (g + 8 * (mt / MTJ)) + 2 * (mt % MTJ);
+    if (ha < G) {
+      OT* op = reinterpret_cast<OT*>(a.out) + (th0 + ha) * D + d_lo;
+      if constexpr (sizeof(OT) == 4) *reinterpret_cast<float2*>(op) = make_float2(o[mt][0] * inv0, o[mt][2] * inv0);
+      else *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[mt][0] * inv0, o[mt][2] * inv0);
     }
-    const float inv0 = l0 > 0.f ? vmul / l0 : 0.f, inv1 = l1 > 0.f ? vmul / l1 : 0.f;
-    const int ha = 8 * u + 2 * tq, hb = ha + 1;
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int d_lo = CH * (g + 8 * (mt / MTJ)) + 2 * (mt % MTJ);
-      if (ha < G) {
-        OT* op = reinterpret_cast<OT*>(a.out) + (th0 + ha) * D + d_lo;
-        if constexpr (sizeof(OT) == 4) *reinterpret_cast<float2*>(op) = make_float2(o[u][mt][0] * inv0, o[u][mt][2] * inv0);
-        else *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[u][mt][0] * inv0, o[u][mt][2] * inv0);
-      }
-      if (hb < G) {
-        OT* op = reinterpret_cast<OT*>(a.out) + (th0 + hb) * D + d_lo;
-        if constexpr (sizeof(OT) == 4) *reinterpret_cast<float2*>(op) = make_float2(o[u][mt][1] * inv1, o[u][mt][3] * inv1);
-        else *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[u][mt][1] * inv1, o[u][mt][3] * inv1);
-      }
+    if (hb < G) {
+      OT* op = reinterpret_cast<OT*>(a.out) + (th0 + hb) * D + d_lo;
+      if constexpr (sizeof(OT) == 4) *reinterpret_cast<float2*>(op) = make_float2(o[mt][1] * inv1, o[mt][3] * inv1);
+      else *reinterpret_cast<__nv_bfloat162*>(op) = __floats2bfloat162_rn(o[mt][1] * inv1, o[mt][3] * inv1);
     }
-    if (a.lse && g == 0) {
-      if (ha < G) a.lse[th0 + ha] = l0 > 0.f ? (m[u][0] + log2f(l0)) * kLn2 : -INFINITY;
-      if (hb < G) a.lse[th0 + hb] = l1 > 0.f ? (m[u][1] + log2f(l1)) * kLn2 : -INFINITY;
-    }
+  }
+  if (a.lse && g == 0) {
+    if (ha < G) a.lse[th0 + ha] = l0 > 0.f ? (m0 + log2f(l0)) * kLn2 : -INFINITY;
+    if (hb < G) a.lse[th0 + hb] = l1 > 0.f ? (m1 + log2f(l1)) * kLn2 : -INFINITY;
   }
 }
 
@@ -328,14 +329,16 @@ template <bool FP8, int D, typename QT, typename OT>
 cudaError_t launch_pf_typed(const AttnArgs& a, float qk, float vmul, cudaStream_t s) {
   const int rows = a.T * a.Hkv;
   const int G = a.Hq / a.Hkv;
-  const size_t smem = (size_t)kPfWarps * pf_stages<FP8, D>() * 32 * Geo<FP8, D>::ROWB;
-  auto go = [&](auto kern) {
+  auto go = [&](auto kern, auto nt_tag) {
+    constexpr int NT = decltype(nt_tag)::value, R = pf_rows<NT>();
+    const size_t smem = (size_t)R * pf_stages<FP8, D, NT>() * 32 * Geo<FP8, D>::ROWB;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     return e != cudaSuccess ? e
-                            : launch_k(kern, dim3((rows + kPfWarps - 1) / kPfWarps), dim3(kPfWarps * 32), smem, s, 1,
-                                       a, qk, vmul, rows);
+                            : launch_k(kern, dim3((rows + R - 1) / R), dim3(R * NT * 32), smem, s, 1, a, qk, vmul,
+                                       rows);
   };
-  return G > 8 ? go(attn_prefill_kernel<FP8, D, QT, OT, 2>) : go(attn_prefill_kernel<FP8, D, QT, OT, 1>);
+  return G > 8 ? go(attn_prefill_kernel<FP8, D, QT, OT, 2>, std::integral_constant<int, 2>())
+               : go(attn_prefill_kernel<FP8, D, QT, OT, 1>, std::integral_constant<int, 1>());
 }
 
 template <bool FP8, int D>
