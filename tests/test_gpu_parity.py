@@ -303,6 +303,40 @@ def test_prefix_hist(case):
             assert int(torch.count_nonzero(h).item()) == 0
 
 
+@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+def test_tensor_parallel_heads(kv):
+    """Tensor parallelism over heads needs no library support: each "rank"
+    calls the decode attention with its slice of query heads, its KV head's
+    cache and the shared selection, and gets its slice of the full output
+    and LSE (summation orders differ with the launch shape, so within a
+    tolerance far inside the parity bounds)."""
+    from indexer_top_sparse_c4_b200 import qsa
+    w = wl.b1_16k(device="cuda", kv_dtype=kv, B=2)
+    step = QSAStep(w)
+    step.run()
+    torch.cuda.synchronize()
+    assert int(step.status.item()) == 0
+    full, full_lse = step.out.float(), step.lse
+    G = w.Hq // w.Hkv
+    for kvh in range(w.Hkv):
+        q = w.q[:, kvh * G:(kvh + 1) * G].contiguous()
+        kp = w.k_pages[:, :, kvh:kvh + 1].contiguous()
+        vp = w.v_pages[:, :, kvh:kvh + 1].contiguous()
+        out = torch.empty((w.T, G, w.D), dtype=step.out.dtype, device="cuda")
+        lse = torch.empty((w.T, G), dtype=torch.float32, device="cuda")
+        ws_bytes = qsa.qsa_sparse_attn_decode_workspace_size(w.T, G, 1, w.D, w.W, kp.dtype)
+        ws = torch.empty((max(ws_bytes, 16),), dtype=torch.uint8, device="cuda")
+        status = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        qsa.qsa_sparse_attn_decode(q, kp, vp, w.page_table, step.tok, step.n_tok, out, workspace=ws,
+                                   k_scale=w.k_scale, v_scale=w.v_scale, q_req=w.q_req, lse=lse,
+                                   dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        ref = full[:, kvh * G:(kvh + 1) * G]
+        assert float((out.float() - ref).abs().max()) <= 4e-3
+        assert float((lse - full_lse[:, kvh * G:(kvh + 1) * G]).abs().max()) <= 1e-4
+
+
 def test_mtp_draft_reuse(oracle):
     w = wl.mtp(device="cuda")
     step = QSAStep(w)
