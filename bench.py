@@ -393,12 +393,7 @@ def gpu_arm(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
         "data": "synthetic",
-        "config": {"workload": w0.name, "B": w0.B, "context": args.context, "Hq": w0.Hq, "Hkv": w0.Hkv,
-                   "D": w0.D, "H_I": w0.H_I, "D_I": w0.D_I, "budget_groups": w0.K,
-                   "kv_storage": "fp8_e4m3 per-tensor scale", "indexer_keys": "fp32, peaked (5% +3 sigma)",
-                   "page_table": "random permutation, page size 64",
-                   "l2": "inputs larger than L2: 256 MiB of indexer keys per step, 2 alternating input sets",
-                   "parallelism": f"dp{ws} (independent request batches)"},
+        "config": decode_config(w0.name, w0.B, args.context, w0.Hq, w0.Hkv, w0.D, w0.H_I, w0.D_I, w0.K, ws),
         "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": round(idx_gbs, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(idx_gbs / peak, 4), "traffic": profiled_traffic(args.context),
@@ -528,6 +523,15 @@ def cpu_baseline(K, seed, seconds):
             f"(262,144 context, K={w.K} groups), all four stages, {el:.1f} s"}
 
 
+def decode_config(name, B, context, Hq, Hkv, D, H_I, D_I, K, ws):
+    """The workload description both arms print."""
+    return {"workload": name, "B": B, "context": context, "Hq": Hq, "Hkv": Hkv, "D": D, "H_I": H_I,
+            "D_I": D_I, "budget_groups": K, "kv_storage": "fp8_e4m3 per-tensor scale",
+            "indexer_keys": "fp32, peaked (5% +3 sigma)", "page_table": "random permutation, page size 64",
+            "l2": "inputs larger than L2: 256 MiB of indexer keys per step, 2 alternating input sets",
+            "parallelism": f"dp{ws} (independent request batches)"}
+
+
 def reference_arm(args):
     ws, rank, local = dist_env()
     if rank != 0:
@@ -547,7 +551,7 @@ def reference_arm(args):
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": 8, "context": 262144, "budget_groups": w.K},
+        "config": decode_config(w.name, 8, 262144, w.Hq, w.Hkv, w.D, w.H_I, w.D_I, w.K, ws),
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": orc.threads_for(w.T),
                          "kind": "oracle", "sample": f"each step: one of the 8 requests "
                          f"(262,144 context, K={w.K} groups), all four stages"},
