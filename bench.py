@@ -411,6 +411,8 @@ def gpu_arm(args):
     }
     if budgets:
         line["other_budgets"] = budgets
+    if args.mtp and ws == 1:
+        line["mtp"] = mtp_summary(device, stream, args.seed, 20)
     if args.prefill and ws == 1:
         line["prefill"] = prefill_summary(device, stream, args.seed, 3)
     if ws == 1 and not args.no_cpu_baseline:
@@ -472,6 +474,54 @@ def prefill_summary(device, stream, seed, reps):
                                 "achieved": round(attn_tf, 1), "peak": peak, "peak_kind": kind,
                                 "unit": "TFLOP/s", "frac": round(attn_tf / peak, 4)},
     }
+
+
+def mtp_summary(device, stream, seed, loops, drafts=2):
+    """The MTP draft loop with index sharing on the B8 x 262,144 FP8 workload:
+    a capture step at p0 (the last token of a block) and `drafts` draft steps
+    at p0 + 1 .. that reuse its selection (plus the group completed since)
+    and only attend.  Two loop sets alternate, so every capture step streams
+    its 256 MiB of indexer keys from HBM; `loops` loops are one CUDA graph."""
+    from indexer_top_sparse_c4_b200 import workloads as wl
+    from indexer_top_sparse_c4_b200.pipeline import QSADraftLoop
+    ctx, B, K = 262144, 8, 512
+    p0 = ((ctx - 4 - drafts) // 4) * 4 + 3   # the last token of a block; p0 + drafts < ctx
+    sets = []
+    for sd in (seed, seed + 1):
+        w = wl.make(f"mtp_b8_262k_fp8_k{K}_draft{drafts}", B=B, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4,
+                    D_I=128, K=K, kv_dtype="fp8", q_dtype="bf16", dist="peaked", pages="perm", seed=sd,
+                    device=device, q_pos=torch.full((B,), p0, dtype=torch.int32),
+                    q_req=torch.arange(B, dtype=torch.int32))
+        sets.append(QSADraftLoop(w, drafts=drafts, seed=sd + 7))
+    with torch.cuda.stream(stream):
+        for i in range(4):
+            sets[i % 2].run()
+        torch.cuda.synchronize()
+        times = {}
+        for name in ("loop", "capture", "draft"):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for i in range(loops):
+                    st = sets[i % 2]
+                    if name == "loop":
+                        st.run()
+                    elif name == "capture":
+                        st.capture.run()
+                    else:
+                        st.draft_step(0)
+            g.replay()
+            times[name] = replay_ms(g) / loops
+            del g
+        for st in sets:  # the capture-only graph leaves the histograms counted up
+            st.capture.prefix_hist.zero_()
+    ok = all(int(st.status.item()) == 0 for st in sets)
+    per_loop = B * (1 + drafts)
+    return {"workload": sets[0].w.name, "B": B, "context": ctx, "capture_pos": p0, "drafts": drafts,
+            "tokens_per_loop": per_loop, "tokens_per_s": round(per_loop / (times["loop"] / 1e3), 1),
+            "ms_per_loop": round(times["loop"], 5),
+            "stages_us": {"capture_step": round(times["capture"] * 1e3, 2),
+                          "draft_step": round(times["draft"] * 1e3, 2)},
+            "device_status_ok": ok}
 
 
 def prefill_arm(args):
@@ -574,6 +624,8 @@ def main(argv=None):
     ap.add_argument("--headline-only", dest="all_budgets", action="store_false")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-mtp", dest="mtp", action="store_false",
+                    help="skip the MTP draft loop (index sharing) line")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false",
                     help="leave out the prefill-chunk summary of the decode line")
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",

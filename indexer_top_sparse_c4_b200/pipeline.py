@@ -97,3 +97,53 @@ class QSAStep:
         self.select(stream)
         self.attention(stream, sm_scale)
         return self.out
+
+
+class QSADraftLoop:
+    """The MTP draft loop with index sharing (TensorRT-LLM
+    "QSASparseAttentionConfig", the MTP index-sharing field): the capture
+    step at p0 scores, selects and attends like any decode step; each of the
+    `drafts` draft steps at p0 + i reuses the captured selection, with the
+    groups completed since p0 appended (qsa_expand_select with capture_pos),
+    and only attends.  The indexer does not run again during the loop.
+
+    Draft step i has one row per capture row (the same request), its own
+    attention query (seeded, the capture query's dtype and shape) and its own
+    token lists and output.  Plumbing only: every stage is a libqsa call."""
+
+    def __init__(self, w: Workload, drafts: int = 2, seed: int = 1):
+        if w.capture_pos is not None:
+            raise ValueError("the capture workload is a plain decode workload")
+        self.w = w
+        self.drafts = drafts
+        self.capture = QSAStep(w)
+        dev = w.q.device
+        g = torch.Generator(device="cpu").manual_seed(seed)
+        T = w.T
+        c0 = w.q_pos // GROUP_TOKENS
+        self.pos = [(w.q_pos + i).contiguous() for i in range(1, drafts + 1)]
+        extra = int((self.pos[-1] // GROUP_TOKENS - c0).max().item())  # groups completed since p0
+        self.W = GROUP_TOKENS * w.K + GROUP_TOKENS + GROUP_TOKENS * max(0, extra)
+        self.q = [torch.randn(w.q.shape, generator=g).to(dtype=w.q.dtype, device=dev) for _ in range(drafts)]
+        self.tok = [torch.empty((T, self.W), dtype=torch.int32, device=dev) for _ in range(drafts)]
+        self.n_tok = [torch.empty((T,), dtype=torch.int32, device=dev) for _ in range(drafts)]
+        self.out = [torch.empty_like(self.capture.out) for _ in range(drafts)]
+        self.lse = [torch.empty_like(self.capture.lse) for _ in range(drafts)]
+        ws = qsa.qsa_sparse_attn_decode_workspace_size(T, w.Hq, w.Hkv, w.D, self.W, w.k_pages.dtype)
+        self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
+        self.status = self.capture.status
+
+    def draft_step(self, i: int, stream=None, sm_scale=0.0):
+        w, cap = self.w, self.capture
+        qsa.qsa_expand_select(cap.sel, cap.n_sel, self.pos[i], self.tok[i], self.n_tok[i],
+                              capture_pos=w.q_pos, dev_status=self.status, stream=stream)
+        qsa.qsa_sparse_attn_decode(self.q[i], w.k_pages, w.v_pages, w.page_table, self.tok[i],
+                                   self.n_tok[i], self.out[i], workspace=self.ws, k_scale=w.k_scale,
+                                   v_scale=w.v_scale, q_req=w.q_req, sm_scale=sm_scale,
+                                   lse=self.lse[i], dev_status=self.status, stream=stream)
+
+    def run(self, stream=None, sm_scale=0.0):
+        self.capture.run(stream, sm_scale)
+        for i in range(self.drafts):
+            self.draft_step(i, stream, sm_scale)
+        return [self.capture.out] + self.out

@@ -347,6 +347,40 @@ def test_mtp_draft_reuse(oracle):
         assert set(range(p0 - 3, p0 + 1)) <= set(tok[t, : host(step.n_tok)[t]].tolist())
 
 
+@pytest.mark.parametrize("ctx,B,kv", [(16384, 2, "bf16"), (262144, 2, "fp8")])
+def test_mtp_draft_loop(oracle, ctx, B, kv):
+    """The draft loop with index sharing: each draft step's token list is the
+    oracle's expansion of the selection captured at p0 (with the groups
+    completed since appended), bit for bit, and its attention matches the
+    oracle on that list.  The capture position is the last token of a block,
+    so every draft step appends the group completed since."""
+    from indexer_top_sparse_c4_b200.pipeline import QSADraftLoop
+    p0 = ((ctx - 6) // 4) * 4 + 3
+    pos = torch.full((B,), p0, dtype=torch.int32)
+    w = wl.make("mtp_capture", B=B, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype=kv,
+                q_dtype="bf16", dist="peaked", pages="perm", device="cuda", q_pos=pos,
+                q_req=torch.arange(B, dtype=torch.int32))
+    loop = QSADraftLoop(w, drafts=2)
+    loop.run()
+    torch.cuda.synchronize()
+    assert int(loop.status.item()) == 0
+    n = {k: host(getattr(w, k)) for k in ("page_table", "q_req", "q_pos")}
+    sel, n_sel = host(loop.capture.sel), host(loop.capture.n_sel)
+    for i in range(loop.drafts):
+        tok_ref, ntok_ref, bad = oracle.expand_select(sel, n_sel, host(loop.pos[i]), loop.W, n["q_pos"])
+        assert bad == 0
+        tok, ntok = host(loop.tok[i]), host(loop.n_tok[i])
+        assert np.array_equal(ntok, ntok_ref) and np.array_equal(tok, tok_ref)
+        for t in range(B):   # the group completed since the capture is in the list
+            assert set(range(p0 - 3, p0 + 1)) <= set(tok[t, :ntok[t]].tolist())
+        kc, vc, pt = compact_pages(w.k_pages, w.v_pages, w.page_table, tok, ntok, n["q_req"])
+        out_ref, lse_ref, sk = oracle.sparse_attn(host(loop.q[i]), kc, vc, pt, tok, ntok, w.k_scale,
+                                                  w.v_scale, q_req=n["q_req"])
+        assert sk == 0
+        mx, mean, rel = attn_errors(out_as_f64(loop.out[i]), out_ref)
+        assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2, (mx, mean, rel)
+
+
 SWEEP = [  # every value of every sweep axis appears at least once
     (4096, 1, (16, 2), 512, "bf16", "ties"),
     (4096, 8, (3, 1), 2048, "fp8", "normal"),
