@@ -37,11 +37,12 @@ using namespace attn;
 
 // ---- decode: one 16-token tile per warp ---------------------------------------
 //
-// The streaming kernel above keeps one or two warps per SM sub-partition busy
-// with a long dependent instruction chain per round; at decode sizes that
-// chain, not HBM, sets the time.  Here every warp owns exactly ONE tile, so a
-// CTA of 4 warps covers one 64-token chunk and there is no softmax state to
-// carry between tiles: K and V go straight into registers, the Q fragments sit
+// A kernel that streams a whole row through one CTA keeps one or two warps per
+// SM sub-partition busy with a long dependent instruction chain per round; at
+// decode sizes that chain, not HBM, sets the time.  Here every warp owns
+// exactly ONE tile, so a CTA of 4 warps covers one 64-token chunk and there is
+// no softmax state to carry between tiles: K and V go straight into registers,
+// the Q fragments sit
 // pre-permuted in shared memory, and each output accumulator is written out
 // right after its single MMA.  That keeps the kernel small enough for four
 // CTAs (16 warps) per SM, which hides the latencies.  Partials are merged per
