@@ -240,8 +240,8 @@ def _fake_hist(scores, q_pos, stride, how):
     return h
 
 
-@pytest.mark.parametrize("case", ["b1_16k", "b4_65k_peaked", "b2_262k_peaked", "b2_65k_normal_k2048",
-                                  "ties", "tiny", "dense_fallback"])
+@pytest.mark.parametrize("case", ["b1_16k", "b4_65k_peaked", "b2_262k_peaked", "b2_262k_odd_stride",
+                                  "b2_65k_normal_k2048", "ties", "tiny", "dense_fallback"])
 def test_prefix_hist(case):
     """The scan's prefix histogram equals the one counted on the host from its
     scores; the Top-K (and the fused expansion) given it returns exactly what
@@ -254,7 +254,7 @@ def test_prefix_hist(case):
         w = wl.b1_16k(device="cuda")
     elif case == "b4_65k_peaked":      # clusters of 2 CTAs per row
         w = wl.b8_262k(device="cuda", B=4, ctx=65536)
-    elif case == "b2_262k_peaked":     # clusters of 8 CTAs per row
+    elif case in ("b2_262k_peaked", "b2_262k_odd_stride"):     # clusters of 8 CTAs per row
         w = wl.b8_262k(device="cuda", B=2)
     elif case == "b2_65k_normal_k2048":
         w = wl.b8_262k(device="cuda", B=2, ctx=65536, K=2048, dist="normal", kv_dtype="bf16")
@@ -264,7 +264,8 @@ def test_prefix_hist(case):
         w = wl.tiny(device="cuda")
     else:
         w = wl.b1_16k(device="cuda", K=8192)
-    step = QSAStep(w, prefix_hist=True)
+    # an odd score-row stride takes the Top-K's scalar score loads
+    step = QSAStep(w, prefix_hist=True, score_stride=65537 if case == "b2_262k_odd_stride" else None)
     step.index_scores()
     torch.cuda.synchronize()
     assert int(step.status.item()) == 0
