@@ -241,7 +241,7 @@ def _fake_hist(scores, q_pos, stride, how):
 
 
 @pytest.mark.parametrize("case", ["b1_16k", "b4_65k_peaked", "b2_262k_peaked", "b2_262k_odd_stride",
-                                  "b2_65k_normal_k2048", "ties", "tiny", "dense_fallback"])
+                                  "b2_65k_normal_k2048", "ties", "tiny", "dense_fallback", "ragged_rows"])
 def test_prefix_hist(case):
     """The scan's prefix histogram equals the one counted on the host from its
     scores; the Top-K (and the fused expansion) given it returns exactly what
@@ -262,6 +262,12 @@ def test_prefix_hist(case):
         w = wl.b8_262k(device="cuda", B=2, ctx=65536, dist="ties")
     elif case == "tiny":
         w = wl.tiny(device="cuda")
+    elif case == "ragged_rows":   # 40 rows of one request, dense and selected rows in one cluster launch
+        pos = np.sort(np.random.default_rng(11).integers(4, 65536, 40)).astype(np.int32)
+        pos[:3] = [5, 1000, 2050]   # c <= K: the dense rows
+        w = wl.make("ragged", B=1, ctx=65536, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="fp8",
+                    q_dtype="bf16", dist="peaked", seed=12, device="cuda", q_pos=pos,
+                    q_req=np.zeros(40, np.int32))
     else:
         w = wl.b1_16k(device="cuda", K=8192)
     # an odd score-row stride takes the Top-K's scalar score loads
