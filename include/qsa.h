@@ -29,7 +29,12 @@
  *    outside the page table, a selected group outside the candidates) is
  *    skipped and ORed into *dev_status as a QSA_DEV_* bit when dev_status is
  *    not NULL.  No kernel traps.  The status word is only ever ORed into;
- *    the caller clears it.
+ *    the caller clears it.  The word is the caller's, one uint32 of device
+ *    memory passed to every call; qsa_get_device_status reads it on the host
+ *    and turns its bits into QSA_ERR_DEVICE_INDEX or QSA_ERR_TIMEOUT.  (The
+ *    "QSA HiSparse" README's offload contract has unsupported configurations
+ *    fail at start-up; a kernel cannot return a code, so errors found on the
+ *    device go through this word instead of aborting the context.)
  *  - Layouts (row-major, innermost last):
  *      indexer query    q_idx        [T, H_I, D_I]          f32 | bf16
  *      indexer weights  w_idx        [T, H_I]               f32
@@ -71,7 +76,13 @@ typedef enum {
   QSA_ERR_INVALID_ARG = 1, /* a null pointer, bad shape, misalignment */
   QSA_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement */
   QSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
-  QSA_ERR_CUDA = 4         /* a CUDA launch or attribute call failed */
+  QSA_ERR_CUDA = 4,        /* a CUDA launch, copy or attribute call failed */
+  QSA_ERR_DEVICE_INDEX = 5, /* qsa_get_device_status: a kernel skipped bad data on
+                               the device (a page, token, group or request id out
+                               of range; any QSA_DEV_* bit but QSA_DEV_TIMEOUT) */
+  QSA_ERR_TIMEOUT = 6      /* qsa_get_device_status: a bounded wait inside a kernel
+                              ran out (QSA_DEV_TIMEOUT); that launch's outputs are
+                              invalid */
 } qsa_status_t;
 
 typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
@@ -110,6 +121,10 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
  * pass leaves the buffer as it is.  Given to the Top-K call that reads these
  * scores, the histogram replaces that call's first radix passes; the Top-K
  * call zeroes it again. */
+/* Workspace of qsa_index_scores: 0 bytes for every supported shape (the scan
+ * and the tensor-core pass keep their state on chip).  Every stage has such a
+ * query so that a caller can size all of them the same way. */
+QSA_API size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride);
 QSA_API qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
                               const int32_t* page_table, int pt_rows, int pt_stride,
@@ -147,6 +162,8 @@ QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint
  * sel entry outside [0, c(p0)) becomes four -1 slots and sets
  * QSA_DEV_BAD_GROUP; a row wider than W is cut at W and sets
  * QSA_DEV_ROW_RANGE.  W >= 4*K + 4 (+4 per group completed since capture). */
+/* Workspace of qsa_expand_select: 0 bytes (one thread per output slot). */
+QSA_API size_t qsa_expand_select_workspace_size(int T, int K, int W);
 QSA_API qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K,
                                const int32_t* q_pos, const int32_t* capture_pos, int T,
                                int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
@@ -195,6 +212,10 @@ QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, con
                                     void* workspace, size_t workspace_bytes,
                                     uint32_t* dev_status, qsa_stream_t stream);
 
+/* Workspace of qsa_sparse_attn_prefill: 0 bytes (each (query, KV head) row is
+ * finished by the warps that stream it). */
+QSA_API size_t qsa_sparse_attn_prefill_workspace_size(int T, int Hq, int Hkv, int D, int W,
+                                                      qsa_dtype_t kv_dt);
 QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void* k_pages,
                                      const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
                                      float v_scale, int num_pages, const int32_t* page_table,
@@ -215,9 +236,12 @@ QSA_API qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, co
  * the library, which every GPU that loads libqsa.so keeps until the process
  * exits; a shape whose scratch (qsa_sparse_attn_decode_workspace_size) is
  * larger is refused with QSA_ERR_WORKSPACE.  The call allocates nothing.
- * The first call on a device looks up that device's copy of the array
- * (cudaGetSymbolAddress, with the device current): make that first call
- * before any stream capture on the device.  Every call shares the one array
+ * The arguments are checked exactly as qsa_sparse_attn_decode checks them,
+ * before the scratch size.  The first call on a device looks up that device's
+ * copy of the array (cudaGetSymbolAddress, with the device current) and keeps
+ * the address: make that first call before any stream capture on the device.
+ * The address belongs to the device's primary context; after cudaDeviceReset,
+ * or from another context, do not call this entry point again on that device.  Every call shares the one array
  * and every kernel overwrites all the scratch it later reads, so nothing
  * needs clearing; but calls whose kernels overlap on the GPU (two streams, or
  * two host threads) race on it -- serialise them. */
@@ -229,13 +253,32 @@ QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
     int Hq, int Hkv, int D, float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
     uint32_t* dev_status, qsa_stream_t stream);
 
+/* Device status query (the boundary's error channel for data the kernels
+ * check on the device; see "Conventions" above).  Waits for `stream` to finish
+ * the work queued so far, reads the caller's status word dev_status and
+ * returns:
+ *   QSA_ERR_TIMEOUT       when QSA_DEV_TIMEOUT is set (it wins over the rest),
+ *   QSA_ERR_DEVICE_INDEX  when any other QSA_DEV_* bit is set,
+ *   QSA_OK                when the word is zero,
+ *   QSA_ERR_CUDA          when the synchronisation or the copy failed
+ *                         (a kernel fault earlier on the stream shows here),
+ *   QSA_ERR_INVALID_ARG   when dev_status is NULL or not 4-byte aligned.
+ * bits_out (host memory, may be NULL) receives the raw word.  clear != 0 sets
+ * the word back to zero after reading it.  Unlike the compute calls, this one
+ * synchronises with the host: call it between steps, never inside a stream
+ * capture. */
+QSA_API qsa_status_t qsa_get_device_status(uint32_t* dev_status, uint32_t* bits_out, int clear,
+                                           qsa_stream_t stream);
+
 /* Human-readable message for the last non-OK status returned on this thread. */
 QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */
 QSA_API const char* qsa_status_name(qsa_status_t s);
 /* ABI version: bumped on any change of the entry points (2: the decode
  * workspace query takes the KV dtype; 3: qsa_topk_expand; 4: the prefix_hist
- * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand). */
+ * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand; 5: the
+ * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
+ * and a workspace query for every stage). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -67,6 +67,16 @@ qsa_status_t check_attn(const void* q, qsa_dtype_t q_dt, const void* k_pages, co
 
 void qsa::set_last_error(const char* msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
 
+qsa_status_t qsa::check_attn_args(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                  const void* v_pages, qsa_dtype_t kv_dt, int num_pages,
+                                  const int32_t* page_table, int pt_rows, int pt_stride,
+                                  const int32_t* tok, const int32_t* n_tok, int W, int T, int Hq,
+                                  int Hkv, int D, void* out, qsa_dtype_t out_dt, float k_scale,
+                                  float v_scale) {
+  return check_attn(q, q_dt, k_pages, v_pages, kv_dt, num_pages, page_table, pt_rows, pt_stride, tok,
+                    n_tok, W, T, Hq, Hkv, D, out, out_dt, k_scale, v_scale);
+}
+
 extern "C" {
 
 const char* qsa_last_error_string(void) { return g_err; }
@@ -78,11 +88,53 @@ const char* qsa_status_name(qsa_status_t s) {
     case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
     case QSA_ERR_WORKSPACE: return "QSA_ERR_WORKSPACE";
     case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+    case QSA_ERR_DEVICE_INDEX: return "QSA_ERR_DEVICE_INDEX";
+    case QSA_ERR_TIMEOUT: return "QSA_ERR_TIMEOUT";
   }
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 4; }
+int qsa_abi_version(void) { return 5; }
+
+size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
+  (void)T; (void)H_I; (void)D_I; (void)score_stride;
+  return 0;
+}
+
+size_t qsa_expand_select_workspace_size(int T, int K, int W) {
+  (void)T; (void)K; (void)W;
+  return 0;
+}
+
+size_t qsa_sparse_attn_prefill_workspace_size(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt) {
+  (void)T; (void)Hq; (void)Hkv; (void)D; (void)W; (void)kv_dt;
+  return 0;
+}
+
+qsa_status_t qsa_get_device_status(uint32_t* dev_status, uint32_t* bits_out, int clear,
+                                   qsa_stream_t stream) {
+  REQUIRE(dev_status != nullptr, "dev_status is NULL");
+  REQUIRE(((uintptr_t)dev_status & 3u) == 0, "dev_status must be 4-byte aligned");
+  const cudaStream_t s = (cudaStream_t)stream;
+  uint32_t bits = 0;
+  // the copy is ordered after the work already queued on the stream
+  qsa_status_t st = cuda_status(cudaMemcpyAsync(&bits, dev_status, sizeof bits, cudaMemcpyDeviceToHost, s),
+                                "qsa_get_device_status: read");
+  if (st == QSA_OK && clear)
+    st = cuda_status(cudaMemsetAsync(dev_status, 0, sizeof bits, s), "qsa_get_device_status: clear");
+  if (st == QSA_OK) st = cuda_status(cudaStreamSynchronize(s), "qsa_get_device_status: stream");
+  if (st != QSA_OK) return st;
+  if (bits_out) *bits_out = bits;
+  if (bits & QSA_DEV_TIMEOUT)
+    return fail(QSA_ERR_TIMEOUT, "a bounded wait inside a kernel ran out (device status 0x%x)", bits);
+  if (bits)
+    return fail(QSA_ERR_DEVICE_INDEX,
+                "a kernel skipped out-of-range data on the device (device status 0x%x: %s%s%s%s%s)",
+                bits, (bits & QSA_DEV_BAD_PAGE) ? "page " : "", (bits & QSA_DEV_BAD_TOKEN) ? "token " : "",
+                (bits & QSA_DEV_BAD_GROUP) ? "group " : "", (bits & QSA_DEV_ROW_RANGE) ? "row-range " : "",
+                (bits & QSA_DEV_BAD_REQUEST) ? "request" : "");
+  return QSA_OK;
+}
 
 qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,
                               const void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,

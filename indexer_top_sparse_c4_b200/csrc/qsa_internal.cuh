@@ -239,5 +239,12 @@ cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, floa
 
 // Sets the message qsa_last_error_string() returns on this thread.
 void set_last_error(const char* msg);
+// The host-side argument checks of the attention calls (shapes, dtypes,
+// pointers, alignment, FP8 scales); QSA_OK or the error, with its message set.
+qsa_status_t check_attn_args(const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages,
+                             qsa_dtype_t kv_dt, int num_pages, const int32_t* page_table, int pt_rows,
+                             int pt_stride, const int32_t* tok, const int32_t* n_tok, int W, int T,
+                             int Hq, int Hkv, int D, void* out, qsa_dtype_t out_dt, float k_scale,
+                             float v_scale);
 
 }  // namespace qsa

@@ -17,17 +17,19 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqsa.so")
 
-QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA = range(5)
+(QSA_OK, QSA_ERR_INVALID_ARG, QSA_ERR_UNSUPPORTED, QSA_ERR_WORKSPACE, QSA_ERR_CUDA,
+ QSA_ERR_DEVICE_INDEX, QSA_ERR_TIMEOUT) = range(7)
 QSA_F32, QSA_BF16, QSA_FP8_E4M3 = 0, 1, 2
 QSA_DEV_BAD_PAGE, QSA_DEV_BAD_TOKEN, QSA_DEV_BAD_GROUP, QSA_DEV_ROW_RANGE = 1, 2, 4, 8
 QSA_DEV_BAD_REQUEST, QSA_DEV_TIMEOUT = 16, 32
 QSA_PREFIX_HIST_BINS = 4096
 
 ENTRY_POINTS = (
-    "qsa_index_scores", "qsa_topk_groups_workspace_size", "qsa_topk_groups",
-    "qsa_expand_select", "qsa_topk_expand", "qsa_sparse_attn_decode_workspace_size",
-    "qsa_sparse_attn_decode",
-    "qsa_sparse_attn_prefill", "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
+    "qsa_index_scores_workspace_size", "qsa_index_scores", "qsa_topk_groups_workspace_size",
+    "qsa_topk_groups", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
+    "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
+    "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
+    "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
 )
 
 
@@ -50,6 +52,14 @@ def lib() -> ctypes.CDLL:
                            "`python -m indexer_top_sparse_c4_b200.build` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.qsa_index_scores_workspace_size.argtypes = [I, I, I, I]
+    L.qsa_index_scores_workspace_size.restype = U
+    L.qsa_expand_select_workspace_size.argtypes = [I, I, I]
+    L.qsa_expand_select_workspace_size.restype = U
+    L.qsa_sparse_attn_prefill_workspace_size.argtypes = [I, I, I, I, I, I]
+    L.qsa_sparse_attn_prefill_workspace_size.restype = U
+    L.qsa_get_device_status.argtypes = [P, P, I, P]
+    L.qsa_get_device_status.restype = I
     L.qsa_index_scores.argtypes = [P, I, P, P, I, I, P, I, I, P, P, I, I, I, P, I, P, P, P]
     L.qsa_topk_groups_workspace_size.argtypes = [I, I, I]
     L.qsa_topk_groups_workspace_size.restype = U
@@ -121,6 +131,32 @@ def qsa_index_scores(q_idx, w_idx, k_idx_pages, page_table, q_pos, scores, q_req
         T, H_I, D_I, _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(dev_status),
         _stream(stream)))
     return scores
+
+
+def qsa_index_scores_workspace_size(T, H_I, D_I, score_stride) -> int:
+    return int(lib().qsa_index_scores_workspace_size(T, H_I, D_I, score_stride))
+
+
+def qsa_expand_select_workspace_size(T, K, W) -> int:
+    return int(lib().qsa_expand_select_workspace_size(T, K, W))
+
+
+def qsa_sparse_attn_prefill_workspace_size(T, Hq, Hkv, D, W, kv_dtype=QSA_BF16) -> int:
+    if isinstance(kv_dtype, torch.dtype):
+        kv_dtype = _dt(torch.empty(0, dtype=kv_dtype))
+    return int(lib().qsa_sparse_attn_prefill_workspace_size(T, Hq, Hkv, D, W, kv_dtype))
+
+
+def qsa_get_device_status(dev_status, clear=False, stream=None):
+    """Read the caller's device status word on the host (synchronises the
+    stream).  Returns (status, bits): QSA_OK, QSA_ERR_DEVICE_INDEX or
+    QSA_ERR_TIMEOUT and the raw word.  Other codes raise QSAError."""
+    bits = ctypes.c_uint32(0)
+    st = lib().qsa_get_device_status(_ptr(dev_status), ctypes.byref(bits), 1 if clear else 0,
+                                     _stream(stream))
+    if st not in (QSA_OK, QSA_ERR_DEVICE_INDEX, QSA_ERR_TIMEOUT):
+        raise QSAError(st, lib().qsa_last_error_string().decode())
+    return st, int(bits.value)
 
 
 def qsa_topk_groups_workspace_size(T, K, score_stride) -> int:

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 4
+    assert L.qsa_abi_version() == 5
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -152,3 +152,31 @@ def test_binding_refuses_to_run_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(qsa, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         qsa.lib()
+
+
+def test_every_stage_has_a_workspace_query(L):
+    """The stages that keep their state on chip report 0 bytes."""
+    from indexer_top_sparse_c4_b200 import qsa
+    assert L.qsa_index_scores_workspace_size(8, 4, 128, 65535) == 0
+    assert L.qsa_index_scores_workspace_size(8192, 4, 128, 16384) == 0
+    assert L.qsa_expand_select_workspace_size(8, 512, 2052) == 0
+    assert L.qsa_sparse_attn_prefill_workspace_size(8192, 24, 2, 256, 2052, 1) == 0
+    for name in ("index_scores", "topk_groups", "expand_select", "sparse_attn_decode",
+                 "sparse_attn_prefill"):
+        assert f"qsa_{name}_workspace_size" in qsa.ENTRY_POINTS
+
+
+def test_status_codes_have_names(L):
+    names = {i: L.qsa_status_name(i).decode() for i in range(7)}
+    assert names[5] == "QSA_ERR_DEVICE_INDEX" and names[6] == "QSA_ERR_TIMEOUT"
+    assert L.qsa_status_name(99).decode() == "QSA_ERR_UNKNOWN"
+
+
+def test_device_status_query_checks_its_pointer(L):
+    """A null or misaligned status word is refused on the host (no copy)."""
+    bits = ctypes.c_uint32(7)
+    assert L.qsa_get_device_status(NULL, ctypes.byref(bits), 0, NULL) == 1
+    assert "NULL" in _err(L)
+    assert L.qsa_get_device_status(ctypes.c_void_p(0x2002), ctypes.byref(bits), 1, NULL) == 1
+    assert "aligned" in _err(L)
+    assert bits.value == 7
