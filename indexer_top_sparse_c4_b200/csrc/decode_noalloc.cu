@@ -14,7 +14,10 @@
 // Host code may not pass the array's name to a kernel (in host code the name
 // is a host-side shadow, not a device address), so the device address is
 // looked up with cudaGetSymbolAddress once per device, with that device
-// current, on the first call made on it.
+// current, on the first call made on it.  The cached address belongs to the
+// device's primary context (the one the CUDA runtime uses); a process that
+// resets the device (cudaDeviceReset) or drives the library from another
+// context must not call this entry point again on that device.
 #include <stdio.h>
 
 #include <mutex>
@@ -60,7 +63,13 @@ qsa_status_t qsa_sparse_attn_decode_noalloc(const void* q, qsa_dtype_t q_dt, con
                                             const int32_t* n_tok, int W, int T, int Hq, int Hkv,
                                             int D, float sm_scale, void* out, qsa_dtype_t out_dt,
                                             float* lse, uint32_t* dev_status, qsa_stream_t stream) {
-  // same checks and kernels as qsa_sparse_attn_decode; only the scratch differs
+  // same checks and kernels as qsa_sparse_attn_decode; only the scratch
+  // differs.  The arguments are checked first, so that a bad or unsupported
+  // shape is reported as such and not as a scratch shortage.
+  const qsa_status_t st = qsa::check_attn_args(q, q_dt, k_pages, v_pages, kv_dt, num_pages, page_table,
+                                               pt_rows, pt_stride, tok, n_tok, W, T, Hq, Hkv, D, out,
+                                               out_dt, k_scale, v_scale);
+  if (st != QSA_OK || T == 0) return st;
   const size_t need = qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv_dt);
   if (need > kScratchFloats * sizeof(float)) {
     char msg[256];
