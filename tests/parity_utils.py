@@ -21,6 +21,14 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.numpy()
 
 
+def values_f64(a: np.ndarray) -> np.ndarray:
+    """The stored values as float64: BF16 bit patterns (uint16, the host form
+    of BF16 tensors) are widened to the floats they encode."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
 def score_bound(q_idx: np.ndarray, w_idx: np.ndarray, khat: np.ndarray, page_table: np.ndarray,
                 q_req: np.ndarray, q_pos: np.ndarray, rows, stride: int) -> np.ndarray:
     """SCORE_REL * sum_h |w_h| sum_d |q_hd k_d| for every (row, group) in rows."""
@@ -31,9 +39,9 @@ def score_bound(q_idx: np.ndarray, w_idx: np.ndarray, khat: np.ndarray, page_tab
             continue
         r = int(q_req[t]) if q_req is not None else t
         pages = page_table[r][: (c + 15) // 16]
-        k = np.abs(khat[pages].reshape(-1, khat.shape[-1])[:c].astype(np.float64))
-        q = np.abs(q_idx[t].astype(np.float64))            # [H, D]
-        out[i, :c] = (np.abs(w_idx[t].astype(np.float64)) @ (q @ k.T)) * SCORE_REL
+        k = np.abs(values_f64(khat[pages].reshape(-1, khat.shape[-1])[:c]))
+        q = np.abs(values_f64(q_idx[t]))                   # [H, D]
+        out[i, :c] = (np.abs(values_f64(w_idx[t])) @ (q @ k.T)) * SCORE_REL
     return out
 
 
