@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "QSA sparse-decode tokens/s @B8×262K FP8 KV; achieved HBM GB/s vs B200 peak"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0   # the B200's nominal HBM3e bandwidth, reported beside the measured peak
 KERNELS_PER_STEP = 3  # index, Top-K with expansion, attention (partials merged inside the clusters)
 
 
@@ -47,22 +48,20 @@ def peak_hbm():
 
 
 def profiled_traffic(context):
-    """DRAM bytes per full-size launch of the indexer scan from the committed ncu
-    summary, or None when the kernel source changed since it was captured (or
-    the workload is not the 262,144-token one the figure is scaled to)."""
+    """DRAM bytes per full-size launch of the indexer scan, from the figure
+    committed beside its ncu summary (profiles/*.json), or None when the
+    kernel source changed since it was captured (or the workload is not the
+    262,144-token one the figure is scaled to)."""
     import hashlib
-    import re
     if context != 262144:
         return None
     try:
-        text = open(os.path.join(ROOT, "profiles", "index_scores_b8_decode_65536_fp8.md")).read()
-        t = re.search(r"traffic_full_size_bytes_per_launch: (\d+)", text)
-        f = re.search(r"source_file: (\S+)", text)
-        h = re.search(r"source_sha256_16: ([0-9a-f]{16})", text)
-        src = open(os.path.join(ROOT, f.group(1)), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != h.group(1):
+        with open(os.path.join(ROOT, "profiles", "index_scores_b8_decode_65536_fp8.json")) as f:
+            rec = json.load(f)
+        src = open(os.path.join(ROOT, rec["source_file"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != rec["source_sha256_16"]:
             return None
-        return int(t.group(1))
+        return int(rec["traffic_full_size_bytes_per_launch"])
     except Exception:
         return None
 
@@ -275,20 +274,25 @@ def pack_inputs(st):
     return dev, host
 
 
-def time_e2e(sets, steps, warmup, stream):
+def time_e2e(sets, steps, warmup, stream, graph=True):
     """Through the public API with host buffers: every step copies its
     query-side inputs from pinned host memory to the device (one packed
     copy), runs the calls and copies the output back to pinned host memory.
     The copies run on two copy streams, so step i+1's inputs go up and step
     i's output comes down while the kernels of step i (i+1) run; events keep
     each buffer safe (a set's inputs are overwritten only after the kernels
-    that read them, its output only after its previous copy-out).  The K
-    timed steps are one captured CUDA graph.  The KV cache and the indexer
-    keys are resident device state."""
+    that read them, its output only after its previous copy-out).  The KV
+    cache and the indexer keys are resident device state.
+    graph=True: the K timed steps are one captured CUDA graph (the calls'
+    host work happens once, at capture).  graph=False: every step issues its
+    copies and library calls from the host inside the timed region (ctypes,
+    argument checks and launches included)."""
     hosts = []
     for st in sets:
-        dev, host = pack_inputs(st)
-        hosts.append((host, dev, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()))
+        if not hasattr(st, "_e2e_buffers"):
+            dev, host = pack_inputs(st)
+            st._e2e_buffers = (host, dev, torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory())
+        hosts.append(st._e2e_buffers)
     h2d = hosts[0][1].numel()
     d2h = hosts[0][2].numel() * hosts[0][2].element_size()
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
@@ -323,20 +327,28 @@ def time_e2e(sets, steps, warmup, stream):
     with torch.cuda.stream(stream):
         steps_on(stream, warmup)
         torch.cuda.synchronize()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            steps_on(stream, steps)
-        g.replay()
-        torch.cuda.synchronize()
-        barrier()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record()
-        g.replay()
-        b.record()
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                steps_on(stream, steps)
+            g.replay()
+            torch.cuda.synchronize()
+            barrier()
+            a.record()
+            g.replay()
+            b.record()
+        else:
+            barrier()
+            torch.cuda.synchronize()
+            a.record()
+            steps_on(stream, steps)
+            b.record()
     torch.cuda.synchronize()
     barrier()
-    del g
+    if graph:
+        del g
     return a.elapsed_time(b), h2d, d2h
 
 
@@ -359,10 +371,13 @@ def gpu_arm(args):
     with ClockSampler(local) as clk:
         total_ms = time_steps(sets, args.steps, args.warmup, stream)
         alone, in_step = time_stages(sets, 40, stream)
-        e2e_ms, h2d, d2h = time_e2e(sets, args.steps, args.warmup, stream)
+        e2e_ms, h2d, d2h = time_e2e(sets, args.steps, args.warmup, stream, graph=True)
+        e2e_eager_ms, _, _ = time_e2e(sets, args.steps, args.warmup, stream, graph=False)
     total_ms = reduce_max(total_ms, device)
     ms = total_ms / args.steps
     e2e_ms = reduce_max(e2e_ms, device)
+    e2e_eager_ms = reduce_max(e2e_eager_ms, device)
+    host_copy = sets[0].w.numpy() if (ws == 1 and not args.no_cpu_baseline) else None
     n_tok_total = int(sets[0].n_tok.sum().item())
     idx_bytes, kv_bytes = algorithmic_bytes(w0, n_tok_total)
     # other budgets, same workload shape, reported beside the headline
@@ -379,8 +394,11 @@ def gpu_arm(args):
             nt = int(sets[0].n_tok.sum().item())
             ib, kb = algorithmic_bytes(sets[0].w, nt)
             peak, _ = peak_hbm()
+            gbs = (ib + kb) / (t / 1e3) / 1e9
             budgets[str(K)] = {"tokens_per_s": round(ws * w0.B / (t / 1e3), 1), "ms_per_step": round(t, 4),
-                               "step_hbm_frac": round((ib + kb) / (t / 1e3) / 1e9 / peak, 4)}
+                               "step_hbm_gbs": round(gbs, 1), "step_hbm_frac": round(gbs / peak, 4),
+                               "step_hbm_frac_nominal": round(gbs / NOMINAL_HBM_GBS, 4),
+                               "bytes_per_step": ib + kb}
     if rank != 0:
         return None
     peak, peak_kind = peak_hbm()
@@ -396,16 +414,35 @@ def gpu_arm(args):
         "config": decode_config(w0.name, w0.B, args.context, w0.Hq, w0.Hkv, w0.D, w0.H_I, w0.D_I, w0.K, ws),
         "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": round(idx_gbs, 1),
                      "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(idx_gbs / peak, 4), "traffic": profiled_traffic(args.context),
-                     "algorithmic_bytes_per_launch": idx_bytes},
+                     "frac": round(idx_gbs / peak, 4), "peak_nominal": NOMINAL_HBM_GBS,
+                     "frac_nominal": round(idx_gbs / NOMINAL_HBM_GBS, 4),
+                     "traffic": profiled_traffic(args.context),
+                     "algorithmic_bytes_per_launch": idx_bytes,
+                     "duration_us": round(alone["index_scores"], 2)},
         "step_hbm": {"achieved": round(step_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(step_gbs / peak, 4), "bytes_per_step": idx_bytes + kv_bytes,
+                     "frac": round(step_gbs / peak, 4), "peak_nominal": NOMINAL_HBM_GBS,
+                     "frac_nominal": round(step_gbs / NOMINAL_HBM_GBS, 4),
+                     "bytes_per_step": idx_bytes + kv_bytes,
                      "indexer_key_bytes": idx_bytes, "selected_kv_bytes": kv_bytes},
+        "attention_hbm": {"bytes_per_launch": kv_bytes,
+                          "duration_us": round(alone["attention"], 2),
+                          "achieved": round(kv_bytes / (alone["attention"] / 1e6) / 1e9, 1),
+                          "frac": round(kv_bytes / (alone["attention"] / 1e6) / 1e9 / peak, 4)},
         "stages_us": {"alone": {n: round(alone[k], 2) for n, k in zip(STAGE_NAMES, STAGES)},
-                      "in_step": {n: round(in_step[k], 2) for n, k in zip(STAGE_NAMES, STAGES)}},
+                      "in_step": {n: round(in_step[k], 2) for n, k in zip(STAGE_NAMES, STAGES)},
+                      "note": "alone: CUDA-event duration per launch from a graph of launches of that "
+                              "stage; in_step: the step graph minus the same graph without the stage "
+                              "(a marginal cost, not a duration)"},
         "e2e": {"value": round(ws * w0.B / (e2e_ms / args.steps / 1e3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(e2e_ms / args.steps, 5)},
+                "ms_per_step": round(e2e_ms / args.steps, 5),
+                "how": "pinned host inputs up, calls, output down, every step; the timed steps "
+                       "replayed from one CUDA graph"},
+        "e2e_eager": {"value": round(ws * w0.B / (e2e_eager_ms / args.steps / 1e3), 1),
+                      "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "ms_per_step": round(e2e_eager_ms / args.steps, 5),
+                      "how": "as e2e, but every step's copies and qsa_* calls are issued from the "
+                             "host inside the timed region (no graph)"},
         "gpu_launches": (KERNELS_PER_STEP + (1 if sets[0].ws_bytes else 0)) * args.steps,
         "clocks": clk.summary(),
     }
@@ -415,8 +452,8 @@ def gpu_arm(args):
         line["mtp"] = mtp_summary(device, stream, args.seed, 20)
     if args.prefill and ws == 1:
         line["prefill"] = prefill_summary(device, stream, args.seed, 3)
-    if ws == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.budget, args.seed, args.cpu_seconds)
+    if host_copy is not None:
+        line["cpu_baseline"] = cpu_baseline(host_copy, w0, args.cpu_seconds)
     return line
 
 
@@ -542,35 +579,59 @@ def prefill_arm(args):
 
 # ---- the oracle on host cores ----------------------------------------------------------
 
-def oracle_sample(K, seed):
-    """One request of the B8 workload (same shapes, recipe and budget), built on
-    the host: the oracle's bounded sample.  Its throughput counts requests, the
-    unit the GPU metric counts."""
+def oracle_inputs(K, seed, context=262144):
+    """Host copies of the B8 workload the GPU arm times (same generator, seed
+    and recipe).  They are drawn on the GPU when there is one, which is
+    where the GPU arm draws them, and copied to the host; the oracle then
+    runs on the host cores only."""
     from indexer_top_sparse_c4_b200 import workloads as wl
-    w = wl.b8_262k(K=K, device="cpu", seed=seed, B=1)
-    return w, w.numpy()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    w = wl.b8_262k(K=K, device=dev, seed=seed, ctx=context)
+    n, k_scale, v_scale = w.numpy(), w.k_scale, w.v_scale
+    del w
+    if dev == "cuda":
+        torch.cuda.empty_cache()
+    return n, k_scale, v_scale
 
 
-def run_oracle_step(orc, n, w):
+def run_oracle_step(orc, n, K, k_scale, v_scale):
+    """One decode step of every request in `n` through the oracle's four stages."""
     return orc.qsa_step(n["q"], n["q_idx"], n["w_idx"], n["k_idx_pages"], n["k_pages"], n["v_pages"],
-                        n["page_table"], n["q_pos"], w.K, w.k_scale, w.v_scale, q_req=n["q_req"])
+                        n["page_table"], n["q_pos"], K, k_scale, v_scale, q_req=n["q_req"])
 
 
-def cpu_baseline(K, seed, seconds):
-    import oracle as orc
-    orc.build()
-    w, n = oracle_sample(K, seed)
+def _time_oracle(orc, n, K, k_scale, v_scale, seconds, min_steps=1):
     t0 = time.perf_counter()
     steps = 0
     while True:
-        run_oracle_step(orc, n, w)
+        run_oracle_step(orc, n, K, k_scale, v_scale)
         steps += 1
         el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return {"value": round(w.B * steps / el, 3), "unit": "tokens/s", "cores": orc.threads_for(w.T),
-            "kind": "oracle", "sample": f"{steps} decode step(s) of one request of the B8 workload "
-            f"(262,144 context, K={w.K} groups), all four stages, {el:.1f} s"}
+        if el >= seconds and steps >= min_steps:
+            return steps, el
+
+
+def cpu_baseline(n, w, seconds):
+    """The oracle as it stands, on the host cores, over the GPU arm's own
+    workload (all 8 requests per step, copied to the host): once with its
+    OpenMP loop over requests on every core it can use, once on one core."""
+    import oracle as orc
+    orc.build()
+    T = int(n["q_pos"].shape[0])
+    host_cores = os.cpu_count() or 1
+    orc.set_max_threads(host_cores)
+    threads = orc.threads_for(T)
+    steps, el = _time_oracle(orc, n, w.K, w.k_scale, w.v_scale, seconds)
+    orc.set_max_threads(1)
+    s1, el1 = _time_oracle(orc, n, w.K, w.k_scale, w.v_scale, seconds / 2)
+    orc.set_max_threads(host_cores)
+    return {"value": round(T * steps / el, 3), "unit": "tokens/s", "cores": threads,
+            "host_cores": host_cores, "kind": "oracle",
+            "sample": f"{steps} decode step(s) of all {T} requests of the GPU arm's workload "
+                      f"(262,144 context, K={w.K} groups), all four stages, {el:.1f} s; the oracle's "
+                      f"OpenMP loop runs over requests, so it uses min({T}, host cores) threads",
+            "single_core": {"value": round(T * s1 / el1, 3), "unit": "tokens/s", "cores": 1,
+                            "sample": f"{s1} step(s), {el1:.1f} s"}}
 
 
 def decode_config(name, B, context, Hq, Hkv, D, H_I, D_I, K, ws):
@@ -583,28 +644,37 @@ def decode_config(name, B, context, Hq, Hkv, D, H_I, D_I, K, ws):
 
 
 def reference_arm(args):
+    """The oracle on the host cores: each timed step is one decode step of all
+    8 requests of the workload the GPU arm times (same generator and seed)."""
     ws, rank, local = dist_env()
     if rank != 0:
         return None
     import oracle as orc
     orc.build()
-    w, n = oracle_sample(args.budget, args.seed)
+    host_cores = os.cpu_count() or 1
+    orc.set_max_threads(host_cores)
+    n, k_scale, v_scale = oracle_inputs(args.budget, rank_seed(args.seed, 0), args.context)
+    T = int(n["q_pos"].shape[0])
     for _ in range(args.warmup):
-        run_oracle_step(orc, n, w)
+        run_oracle_step(orc, n, args.budget, k_scale, v_scale)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        run_oracle_step(orc, n, w)
+        run_oracle_step(orc, n, args.budget, k_scale, v_scale)
     el = time.perf_counter() - t0
-    value = w.B * args.steps / el
+    value = T * args.steps / el
+    threads = orc.threads_for(T)
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
         "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": decode_config(w.name, 8, 262144, w.Hq, w.Hkv, w.D, w.H_I, w.D_I, w.K, ws),
-        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": orc.threads_for(w.T),
-                         "kind": "oracle", "sample": f"each step: one of the 8 requests "
-                         f"(262,144 context, K={w.K} groups), all four stages"},
+        "config": decode_config(f"b8_decode_{args.context // 1024}k_fp8_k{args.budget}", T, args.context,
+                                16, 2, 256, 4, 128, args.budget, ws),
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads,
+                         "host_cores": host_cores, "kind": "oracle",
+                         "sample": f"each step: all {T} requests ({args.context:,} context, "
+                                   f"K={args.budget} groups), all four stages; the oracle's OpenMP "
+                                   f"loop runs over requests"},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }

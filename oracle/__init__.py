@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
                                          I, I, F, P, P]
         _lib.orc_threads_for.restype = I
         _lib.orc_threads_for.argtypes = [I]
+        _lib.orc_set_max_threads.restype = None
+        _lib.orc_set_max_threads.argtypes = [I]
     return _lib
 
 
@@ -97,6 +99,11 @@ def e4m3_to_f64(code: int) -> float:
 
 def threads_for(T: int) -> int:
     return lib().orc_threads_for(T)
+
+
+def set_max_threads(n: int) -> None:
+    """Cap the OpenMP threads of the oracle's loops over query tokens."""
+    lib().orc_set_max_threads(int(n))
 
 
 def index_scores(q_idx, w_idx, k_idx_pages, page_table, q_pos, q_req=None, score_stride=None):

@@ -51,6 +51,14 @@ static double load_val(const void* base, int dt, long idx) {
   }
 }
 
+void orc_set_max_threads(int n) {
+#ifdef _OPENMP
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 int orc_threads_for(int T) {
 #ifdef _OPENMP
   int n = omp_get_max_threads();

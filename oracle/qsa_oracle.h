@@ -92,6 +92,9 @@ long orc_sparse_attn(const void* q, int q_dt, const void* k_pages,
 
 /* Threads the OpenMP loops over query tokens use for a row count of T. */
 int orc_threads_for(int T);
+/* Caps the threads of those loops (the host's core count by default); used to
+ * time the oracle on one core.  Changes no result. */
+void orc_set_max_threads(int n);
 
 #ifdef __cplusplus
 }
