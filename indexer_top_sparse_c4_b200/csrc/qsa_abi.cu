@@ -50,6 +50,8 @@ qsa_status_t check_attn(const void* q, qsa_dtype_t q_dt, const void* k_pages, co
   REQUIRE(W >= 1, "W must be >= 1 (got %d)", W);
   REQUIRE(num_pages >= 1 && pt_rows >= 1 && pt_stride >= 1,
           "num_pages, pt_rows and pt_stride must be >= 1");
+  SUPPORT(num_pages <= (1 << 25), "num_pages = %d exceeds the %d pages (2^31 token rows) a cache may hold",
+          num_pages, 1 << 25);
   REQUIRE(q_dt == QSA_F32 || q_dt == QSA_BF16, "q dtype must be F32 or BF16");
   REQUIRE(kv_dt == QSA_F32 || kv_dt == QSA_BF16 || kv_dt == QSA_FP8_E4M3, "bad KV dtype");
   REQUIRE(out_dt == QSA_F32 || out_dt == QSA_BF16, "out dtype must be F32 or BF16");

@@ -206,10 +206,18 @@ struct AttnArgs {
 // How a decode call is spread over the GPU: clusters of `cl` CTAs per
 // (query, KV head) merged on chip, and `s` cluster groups whose partial
 // (o, max, sum) go through the workspace to the combine kernel when s > 1.
+// Plan of the decode kernel that spreads each (query, KV head) row over S
+// CTAs of C token slots each; with S > 1 the combine kernel merges the S
+// partials of a row.
+struct GatherPlan {
+  int S, C;
+};
 struct DecodePlan {
   int cl, s;
   bool stream;   // tensor-core path: one CTA streams a whole row (no split)
   bool cluster;  // tensor-core path: one cluster of cl CTAs per row, merged on chip
+  bool gather = false;  // tensor-core path: the gather kernel with plan gp; s = gp.S partials per row
+  GatherPlan gp{1, 16};
 };
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
@@ -234,6 +242,13 @@ cudaError_t launch_sparse_attn_cluster(const AttnArgs& a, float qk_scale_log2, f
 // warp, attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on
 // chip, cluster groups merged by the combine kernel.
 int attn_tile_tokens();
+// Decode kernel for few rows on every SM: rows split into chunks of one CTA
+// each (one wave, one CTA per SM), token rows resolved once per chunk, K/V
+// streamed through per-slot cp.async rings (sparse_attn_gather.cu).
+bool attn_gather_supported(const AttnArgs& a);
+GatherPlan attn_gather_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
+cudaError_t launch_sparse_attn_gather(const AttnArgs& a, float qk_scale_log2, float vmul, const GatherPlan& p,
+                                      void* ws, cudaStream_t s);
 cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                     int s, void* ws, cudaStream_t stream);
 

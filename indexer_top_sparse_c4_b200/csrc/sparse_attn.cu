@@ -297,7 +297,13 @@ DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv
   probe.Hq = Hq;
   probe.Hkv = Hkv > 0 ? Hkv : 1;
   DecodePlan p{1, 1, false, false};
-  if (attn_mma_supported(probe)) {
+  if (attn_gather_supported(probe) && T * probe.Hkv < 148) {
+    // few (query, KV head) rows: every row spread over CTAs on all SMs, their
+    // partials merged by the combine kernel
+    p.gather = true;
+    p.gp = attn_gather_plan(T, Hq, probe.Hkv, D, W, kv_dt);
+    p.s = p.gp.S;
+  } else if (attn_mma_supported(probe)) {
     const int halves = probe.Hq / probe.Hkv > 8 ? 2 : 1;  // CTAs per KV head
     const int ctas_per_chunk = T * probe.Hkv * halves;
     int cl = 8;  // the largest cluster that keeps every row's cluster resident at once
@@ -343,7 +349,9 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   sc.qk = (float)(scale * 1.4426950408889634 * (fp8 ? (double)a.k_scale : 1.0));
   sc.vmul = fp8 ? a.v_scale : 1.f;
   cudaError_t e;
-  if (attn_mma_supported(a)) {
+  if (plan.gather) {
+    e = launch_sparse_attn_gather(a, sc.qk, sc.vmul, plan.gp, ws, s);
+  } else if (attn_mma_supported(a)) {
     e = plan.stream    ? launch_sparse_attn_prefill_rows(a, sc.qk, sc.vmul, s)
         : plan.cluster ? launch_sparse_attn_cluster(a, sc.qk, sc.vmul, plan.cl, s)
                        : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);

@@ -135,10 +135,11 @@ def test_attention_validation(L, fn):
 
 
 def test_decode_workspace_is_checked(L):
-    # many rows (prefill-sized T) and rows one cluster covers need no
-    # workspace; rows split across cluster groups do
+    # many (query, KV head) rows (prefill-sized T) need no workspace; a decode
+    # batch spreads each row over several CTAs whose partials go through it
     assert L.qsa_sparse_attn_decode_workspace_size(8192, 24, 2, 256, 2052, 1) == 0
-    assert L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 2052, 1) == 0
+    need = L.qsa_sparse_attn_decode_workspace_size(8, 16, 2, 256, 2052, 2)
+    assert need > 0 and need == 8 * 16 * 9 * (256 + 2) * 4   # 9 chunks per row: 144 CTAs
     need = L.qsa_sparse_attn_decode_workspace_size(1, 16, 2, 256, 8196, 1)
     assert need > 0
     ok = ctypes.c_void_p(0x10000)

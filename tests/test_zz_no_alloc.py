@@ -47,8 +47,8 @@ def test_noalloc_matches_workspace_decode_on_two_calls(lib):
     call's leftover partials by the second would change its output."""
     from indexer_top_sparse_c4_b200 import workloads as wl
     shapes = [
-        lambda: wl.b1_16k(device="cuda", seed=11, B=2, kv_dtype="fp8", K=4096),   # 16,388 slots
-        lambda: wl.b1_16k(device="cuda", seed=12, K=2048),                         # 8,196 slots
+        lambda: wl.b1_16k(device="cuda", seed=11, B=2, kv_dtype="fp8", K=4096),   # 4 rows of 16,388 slots
+        lambda: wl.b1_16k(device="cuda", seed=12, K=512),                          # 2 rows of 2,052 slots
     ]
     needs = []
     for make in shapes:
@@ -64,8 +64,9 @@ def test_noalloc_matches_workspace_decode_on_two_calls(lib):
 
 
 def test_noalloc_refuses_shapes_beyond_its_buffer(lib):
-    # 64 queries x 16 heads x many split partials of 256 floats exceed 32 MiB
-    T, Hq, Hkv, D, W = 64, 16, 2, 256, 8196
+    # 2 queries x 16 heads x 1,024 chunk partials (rows of 2^20 slots, 1,024
+    # slots per chunk) of 258 floats exceed 32 MiB
+    T, Hq, Hkv, D, W = 2, 16, 1, 256, 1 << 20
     assert lib.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, torch.uint8) > 32 * 1024 * 1024
     q = torch.zeros((T, Hq, D), dtype=torch.bfloat16, device="cuda")
     kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")  # FP8 codes
@@ -80,7 +81,7 @@ def test_noalloc_refuses_shapes_beyond_its_buffer(lib):
 def test_noalloc_reports_bad_arguments_before_the_scratch_size(lib):
     """A shape that is invalid (Hq not a multiple of Hkv) and would also need
     more scratch than the buffer holds is refused as an invalid argument."""
-    T, Hq, Hkv, D, W = 64, 15, 2, 256, 8196
+    T, Hq, Hkv, D, W = 2, 15, 2, 256, 1 << 20
     q = torch.zeros((T, Hq, D), dtype=torch.bfloat16, device="cuda")
     kv = torch.zeros((1, 64, Hkv, D), dtype=torch.uint8, device="cuda")
     pt = torch.zeros((T, 1), dtype=torch.int32, device="cuda")
