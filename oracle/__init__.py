@@ -63,6 +63,10 @@ def lib() -> ctypes.CDLL:
         _lib.orc_sparse_attn.restype = L
         _lib.orc_sparse_attn.argtypes = [P, I, P, P, I, F, F, I, P, I, P, P, P, I, I, I,
                                          I, I, F, P, P]
+        _lib.orc_indexer_project.restype = L
+        _lib.orc_indexer_project.argtypes = [P, I, P, I, I, I, I, P]
+        _lib.orc_compress_keys.restype = L
+        _lib.orc_compress_keys.argtypes = [P, I, P, P, P, P, I, P, I, I, P, I, I]
         _lib.orc_threads_for.restype = I
         _lib.orc_threads_for.argtypes = [I]
         _lib.orc_set_max_threads.restype = None
@@ -180,6 +184,44 @@ def sparse_attn(q, k_pages, v_pages, page_table, tok, n_tok, k_scale=1.0, v_scal
     if rc < 0:
         raise ValueError(f"orc_sparse_attn failed ({rc})")
     return out, lse, int(rc)
+
+
+def indexer_project(x, w):
+    """Before stage 1: y [T,N] float32 = x [T,H] . w [N,H]^T (float32 or BF16
+    bit patterns as uint16), accumulated in double."""
+    x = np.ascontiguousarray(x)
+    w = np.ascontiguousarray(w)
+    T, H = x.shape
+    N, H2 = w.shape
+    assert H2 == H
+    y = np.empty((T, N), np.float32)
+    rc = lib().orc_indexer_project(_ptr(x), _dt_of(x), _ptr(w), _dt_of(w), T, H, N, _ptr(y))
+    if rc < 0:
+        raise ValueError(f"orc_indexer_project failed ({rc})")
+    return y
+
+
+def compress_keys(k_tok, g_id, wphi, k_idx_pages, page_table, g_req=None, bias=None):
+    """Before stage 1: the C4 compressed-key write.  k_tok [n,4,D_I] float32
+    token keys of n completed groups; writes each group's compressed key into
+    k_idx_pages (float32, or uint16 BF16 bit patterns) IN PLACE through the
+    page table.  Returns the count of skipped groups."""
+    k_tok = _c(k_tok, np.float32)
+    n, four, D_I = k_tok.shape
+    assert four == GROUP_TOKENS
+    assert k_idx_pages.flags.c_contiguous and k_idx_pages.shape[1:] == (PAGE_GROUPS, D_I)
+    wphi = _c(wphi, np.float32)
+    assert wphi.shape == (D_I, GROUP_TOKENS * D_I)
+    b = None if bias is None else _c(bias, np.float32)
+    pt = _c(page_table, np.int32)
+    gid = _c(g_id, np.int32)
+    gr = None if g_req is None else _c(g_req, np.int32)
+    rc = lib().orc_compress_keys(_ptr(k_tok), n, _ptr(gr), _ptr(gid), _ptr(wphi), _ptr(b), D_I,
+                                 _ptr(k_idx_pages), _dt_of(k_idx_pages), k_idx_pages.shape[0], _ptr(pt),
+                                 pt.shape[0], pt.shape[1])
+    if rc < 0:
+        raise ValueError(f"orc_compress_keys failed ({rc})")
+    return int(rc)
 
 
 def qsa_step(q, q_idx, w_idx, k_idx_pages, k_pages, v_pages, page_table, q_pos, K,

@@ -277,3 +277,60 @@ long orc_sparse_attn(const void* q, int q_dt, const void* k_pages,
   }
   return skipped;
 }
+
+/* ---- before stage 1: the indexer projection --------------------------------- */
+
+long orc_indexer_project(const void* x, int x_dt, const void* w, int w_dt, int T, int H, int N,
+                         float* y) {
+  if (T < 0 || H < 1 || N < 1) return -1;
+  if ((x_dt != ORC_F32 && x_dt != ORC_BF16) || (w_dt != ORC_F32 && w_dt != ORC_BF16)) return -2;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(orc_threads_for(T))
+  for (int t = 0; t < T; ++t)
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += load_val(x, x_dt, (long)t * H + h) * load_val(w, w_dt, (long)n * H + h);
+      y[(long)t * N + n] = (float)acc;
+    }
+  return 0;
+}
+
+/* ---- before stage 1: the C4 compressed-key write ----------------------------- */
+
+/* bfloat16 bits of a float, round to nearest even (finite inputs). */
+static uint16_t f32_to_bf16_rne(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  const uint32_t lsb = (u >> 16) & 1u;
+  u += 0x7FFFu + lsb;
+  return (uint16_t)(u >> 16);
+}
+
+long orc_compress_keys(const float* k_tok, int n_groups, const int32_t* g_req, const int32_t* g_id,
+                       const float* wphi, const float* bias, int D_I, void* k_idx_pages, int k_dt,
+                       int num_pages, const int32_t* page_table, int pt_rows, int pt_stride) {
+  if (n_groups < 0 || D_I < 1 || pt_rows < 1 || pt_stride < 1) return -1;
+  if (k_dt != ORC_F32 && k_dt != ORC_BF16) return -2;
+  long skipped = 0;
+  for (int i = 0; i < n_groups; ++i) {
+    const int r = g_req ? g_req[i] : 0;
+    const int g = g_id[i];
+    if (r < 0 || r >= pt_rows || g < 0 || g / ORC_PAGE_GROUPS >= pt_stride) { ++skipped; continue; }
+    const int page = page_table[(long)r * pt_stride + g / ORC_PAGE_GROUPS];
+    if (page < 0 || page >= num_pages) { ++skipped; continue; }
+    const long row = ((long)page * ORC_PAGE_GROUPS + g % ORC_PAGE_GROUPS) * D_I;
+    /* khat[d] = bias[d] + sum over the group's four tokens j and dims e of
+       wphi[d][j * D_I + e] * k_tok[i][j][e] */
+    for (int d = 0; d < D_I; ++d) {
+      double acc = bias ? (double)bias[d] : 0.0;
+      for (int j = 0; j < ORC_GROUP_TOKENS; ++j)
+        for (int e = 0; e < D_I; ++e)
+          acc += (double)wphi[((long)d * ORC_GROUP_TOKENS + j) * D_I + e] *
+                 (double)k_tok[((long)i * ORC_GROUP_TOKENS + j) * D_I + e];
+      const float v = (float)acc;
+      if (k_dt == ORC_F32) ((float*)k_idx_pages)[row + d] = v;
+      else ((uint16_t*)k_idx_pages)[row + d] = f32_to_bf16_rne(v);
+    }
+  }
+  return skipped;
+}

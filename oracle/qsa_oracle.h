@@ -90,6 +90,28 @@ long orc_sparse_attn(const void* q, int q_dt, const void* k_pages,
                      const int32_t* n_tok, int W, int T, int Hq, int Hkv, int D,
                      float sm_scale, double* out, double* lse);
 
+/* Indexer projection (the step before stage 1): y[t][n] = sum_h x[t][h] *
+ * w[n][h] for x [T,H] and w [N,H] (F32 or BF16), accumulated in double and
+ * rounded once to float.  Rows of w stack the indexer query heads (H_I*D_I),
+ * the head weights (H_I) and the token key (D_I).  Returns 0, or a negative
+ * value on an argument error. */
+long orc_indexer_project(const void* x, int x_dt, const void* w, int w_dt, int T, int H, int N,
+                         float* y);
+
+/* C4 compressed-key write (the step before stage 1).  For completed group i
+ * (request g_req[i], NULL: request 0; group id g_id[i]) with token keys
+ * k_tok[i][0..3][0..D_I) (f32):
+ *   khat[d] = bias[d] + sum_{j<4} sum_{e<D_I} wphi[d][j*D_I + e] * k_tok[i][j][e]
+ * (wphi [D_I][4*D_I] f32, bias [D_I] f32 or NULL), accumulated in double,
+ * rounded once to float (then to bfloat16, round to nearest even, for BF16
+ * storage) and written to row g%16 of page page_table[req][g/16] of
+ * k_idx_pages [num_pages,16,D_I] (k_dt F32 or BF16).  A group whose request,
+ * logical page or physical page is out of range is skipped and counted.
+ * Returns the count, or a negative value on an argument error. */
+long orc_compress_keys(const float* k_tok, int n_groups, const int32_t* g_req, const int32_t* g_id,
+                       const float* wphi, const float* bias, int D_I, void* k_idx_pages, int k_dt,
+                       int num_pages, const int32_t* page_table, int pt_rows, int pt_stride);
+
 /* Threads the OpenMP loops over query tokens use for a row count of T. */
 int orc_threads_for(int T);
 /* Caps the threads of those loops (the host's core count by default); used to

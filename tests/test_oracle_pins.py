@@ -421,3 +421,94 @@ def test_sm_scale_default_is_inverse_sqrt_d(oracle):
     b, _, _ = oracle.sparse_attn(n["q"], n["k_pages"], n["v_pages"], n["page_table"], tok, np.array([3]),
                                  sm_scale=1 / math.sqrt(64))
     assert np.array_equal(a, b)
+
+
+# ---- before stage 1: indexer projection and the C4 compressed-key write ----------
+
+def _bf16_bits(a):
+    return torch.tensor(a, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_projection_hand_worked(oracle):
+    """y = x . w^T worked by hand: x = [[1, 2], [3, 4]], w rows (1, 0),
+    (0.5, -1), (2, 2) give [[1, -1.5, 6], [3, -2.5, 14]] (every value exact in
+    BF16 and FP32)."""
+    x = np.array([[1, 2], [3, 4]], np.float32)
+    w = np.array([[1, 0], [0.5, -1], [2, 2]], np.float32)
+    want = np.array([[1, -1.5, 6], [3, -2.5, 14]], np.float32)
+    assert np.array_equal(oracle.indexer_project(x, w), want)
+    assert np.array_equal(oracle.indexer_project(_bf16_bits(x), _bf16_bits(w)), want)
+
+
+def test_projection_is_the_matrix_product(oracle):
+    """Random BF16 inputs: equal, after one rounding, to the float64 matrix
+    product of the decoded values (numpy's routine, not the oracle's loop)."""
+    g = torch.Generator().manual_seed(2)
+    x = torch.randn((5, 96), generator=g).to(torch.bfloat16)
+    w = torch.randn((7, 96), generator=g).to(torch.bfloat16)
+    want = (x.double().numpy() @ w.double().numpy().T).astype(np.float32)
+    got = oracle.indexer_project(x.view(torch.int16).numpy().view(np.uint16),
+                                 w.view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(got, want)
+
+
+def _pages(num_pages, D_I, dt):
+    if dt == "f32":
+        return np.full((num_pages, 16, D_I), 7.0, np.float32)
+    return np.full((num_pages, 16, D_I), 0x40E0, np.uint16)     # 7.0 in BF16
+
+
+def test_compression_mean_pooling_and_selection(oracle):
+    """wphi = [I/4, I/4, I/4, I/4] pools the group's four token keys into their
+    mean; wphi = [0, I, 0, 0] selects the second token's key; a bias adds."""
+    D_I = 8
+    rng = np.random.default_rng(3)
+    k_tok = rng.integers(-8, 8, size=(3, 4, D_I)).astype(np.float32)   # small integers: exact sums
+    I = np.eye(D_I, dtype=np.float32)
+    pt = np.array([[2, 0, 1]], np.int32)
+    gid = np.array([0, 17, 40], np.int32)     # logical pages 0, 1, 2 -> physical 2, 0, 1
+    mean_w = np.concatenate([I / 4] * 4, axis=1)
+    pages = _pages(3, D_I, "f32")
+    assert oracle.compress_keys(k_tok, gid, mean_w, pages, pt) == 0
+    assert np.array_equal(pages[2, 0], k_tok[0].mean(axis=0))
+    assert np.array_equal(pages[0, 1], k_tok[1].mean(axis=0))
+    assert np.array_equal(pages[1, 8], k_tok[2].mean(axis=0))
+    sel_w = np.concatenate([0 * I, I, 0 * I, 0 * I], axis=1)
+    bias = np.arange(D_I, dtype=np.float32)
+    assert oracle.compress_keys(k_tok, gid, sel_w, pages, pt, bias=bias) == 0
+    assert np.array_equal(pages[2, 0], k_tok[0, 1] + bias)
+    assert np.array_equal(pages[1, 8], k_tok[2, 1] + bias)
+
+
+def test_compression_writes_only_its_rows(oracle):
+    """Each group lands in row g % 16 of page table[req][g // 16]; every other
+    row keeps its contents; out-of-range requests and pages are skipped."""
+    D_I = 4
+    k_tok = np.ones((4, 4, D_I), np.float32)
+    wphi = np.concatenate([np.eye(D_I, dtype=np.float32)] * 4, axis=1)   # sum of the four keys
+    pt = np.array([[1, 3], [0, 99]], np.int32)
+    gid = np.array([5, 16, 18, 20], np.int32)
+    req = np.array([0, 0, 1, 1], np.int32)    # (1, 18) and (1, 20) -> page 99: out of range
+    pages = _pages(4, D_I, "f32")
+    before = pages.copy()
+    assert oracle.compress_keys(k_tok, gid, wphi, pages, pt, g_req=req) == 2
+    written = {(1, 5), (3, 0)}
+    for p in range(4):
+        for r in range(16):
+            if (p, r) in written:
+                assert np.all(pages[p, r] == 4.0)
+            else:
+                assert np.array_equal(pages[p, r], before[p, r])
+
+
+def test_compression_bf16_storage_rounds_to_nearest_even(oracle):
+    """BF16 storage keeps 8 significant bits: 1 + 2^-8 is a tie and rounds to
+    1 (even), 1 + 3 * 2^-9 rounds up to 1 + 2^-7, -(2 + 2^-6) is exact."""
+    D_I = 4
+    k_tok = np.zeros((1, 4, D_I), np.float32)
+    k_tok[0, 0] = [1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, -(2 + 2.0 ** -6), 0.5]
+    wphi = np.concatenate([np.eye(D_I, dtype=np.float32)] + [np.zeros((D_I, D_I), np.float32)] * 3, axis=1)
+    pages = _pages(1, D_I, "bf16")
+    oracle.compress_keys(k_tok, np.array([3], np.int32), wphi, pages, np.zeros((1, 1), np.int32))
+    got = torch.from_numpy(pages[0, 3].view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    assert list(got) == [1.0, 1 + 2.0 ** -7, -(2 + 2.0 ** -6), 0.5]
