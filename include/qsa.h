@@ -97,6 +97,45 @@ typedef enum { QSA_F32 = 0, QSA_BF16 = 1, QSA_FP8_E4M3 = 2 } qsa_dtype_t;
 #define QSA_DEV_TIMEOUT 32u   /* a bounded wait inside a kernel ran out (the
                                  kernel stopped early; its outputs are invalid) */
 
+/* Before stage 1 -- the indexer projection (a reading fixed by this library:
+ * "QSA in brief" names a learned indexer, not its layers).  y[t, n] =
+ * sum_h x[t, h] * w[n, h] in FP32 for hidden states x [T, H] and weights
+ * w [N, H] (each F32 or BF16, 16-byte aligned, H a multiple of 8); y [T, N]
+ * FP32, row-major.  Stacking w = [W_q; W_w; W_k] ([H_I*D_I + H_I + D_I, H])
+ * gives every token's indexer query (y[t, 0 .. H_I*D_I)), head weights
+ * (next H_I) and token key (last D_I) in one call.  A few tokens (decode)
+ * take a GEMV that reads w once; BF16 x and w with T >= 128 and H a multiple
+ * of 64 take a tcgen05 GEMM (TMA-fed tiles, TMEM accumulators).
+ * workspace: none (qsa_indexer_project_workspace_size returns 0). */
+QSA_API size_t qsa_indexer_project_workspace_size(int T, int H, int N);
+QSA_API qsa_status_t qsa_indexer_project(const void* x, qsa_dtype_t x_dt, const void* w, qsa_dtype_t w_dt, int T,
+                                         int H, int N, float* y, uint32_t* dev_status, qsa_stream_t stream);
+
+/* Before stage 1 -- the C4 compressed-key write ("QSA in brief": the indexer
+ * keys are compressed over four-token blocks; "QSA HiSparse", entry-point
+ * table: the backend's prefill writes; the compression itself is a reading
+ * fixed by this library).  For each of n_groups completed groups i, with
+ * token keys k_tok[(4*i + j) * tok_stride + e] (j = 0..3 the group's tokens
+ * in order, e < D_I; FP32):
+ *   khat[d] = bias[d] + sum_{j<4} sum_{e<D_I} wphi[d * 4*D_I + j*D_I + e] * k_tok[...]
+ * (wphi [D_I, 4*D_I] FP32; bias [D_I] FP32 or NULL), written to row
+ * g_id[i] % 16 of page page_table[g_req[i]][g_id[i] / 16] of k_idx_pages
+ * [num_pages, 16, D_I] in k_dt (F32, or BF16 rounded to nearest even).
+ * g_req NULL: every group belongs to request 0.  A request id outside
+ * [0, pt_rows) sets QSA_DEV_BAD_REQUEST, a group id < 0 or beyond the page
+ * table QSA_DEV_BAD_GROUP, a physical page outside [0, num_pages)
+ * QSA_DEV_BAD_PAGE; such groups are not written.  Nothing else in
+ * k_idx_pages changes.  D_I in {32, 64, 128}.  With tok_stride the rows of
+ * qsa_indexer_project's output can be read in place (k_tok = y + H_I*D_I +
+ * H_I, tok_stride = N, four consecutive tokens per group).
+ * workspace: none (qsa_compress_keys_workspace_size returns 0). */
+QSA_API size_t qsa_compress_keys_workspace_size(int n_groups, int D_I);
+QSA_API qsa_status_t qsa_compress_keys(const float* k_tok, int tok_stride, int n_groups, const int32_t* g_req,
+                                       const int32_t* g_id, const float* wphi, const float* bias, int D_I,
+                                       void* k_idx_pages, qsa_dtype_t k_dt, int num_pages,
+                                       const int32_t* page_table, int pt_rows, int pt_stride,
+                                       uint32_t* dev_status, qsa_stream_t stream);
+
 /* Width of one row of the optional prefix histogram passed from stage 1 to
  * stage 2 (prefix_hist below): one uint32 count per value of the top 12 bits
  * of a score's order key.  The order key of a float is its bit pattern with
@@ -278,7 +317,8 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * workspace query takes the KV dtype; 3: qsa_topk_expand; 4: the prefix_hist
  * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand; 5: the
  * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
- * and a workspace query for every stage). */
+ * and a workspace query for every stage; 6: qsa_indexer_project and
+ * qsa_compress_keys). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

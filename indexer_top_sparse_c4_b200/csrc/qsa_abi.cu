@@ -96,7 +96,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 5; }
+int qsa_abi_version(void) { return 6; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -136,6 +136,46 @@ qsa_status_t qsa_get_device_status(uint32_t* dev_status, uint32_t* bits_out, int
                 (bits & QSA_DEV_BAD_GROUP) ? "group " : "", (bits & QSA_DEV_ROW_RANGE) ? "row-range " : "",
                 (bits & QSA_DEV_BAD_REQUEST) ? "request" : "");
   return QSA_OK;
+}
+
+size_t qsa_indexer_project_workspace_size(int T, int H, int N) {
+  (void)T; (void)H; (void)N;
+  return 0;
+}
+
+qsa_status_t qsa_indexer_project(const void* x, qsa_dtype_t x_dt, const void* w, qsa_dtype_t w_dt, int T, int H,
+                                 int N, float* y, uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(T >= 0 && H >= 1 && N >= 1, "need T >= 0, H >= 1, N >= 1 (got %d, %d, %d)", T, H, N);
+  REQUIRE(x_dt == QSA_F32 || x_dt == QSA_BF16, "x dtype must be F32 or BF16");
+  REQUIRE(w_dt == QSA_F32 || w_dt == QSA_BF16, "w dtype must be F32 or BF16");
+  SUPPORT(H % 8 == 0, "the hidden size H = %d must be a multiple of 8", H);
+  if (T == 0) return QSA_OK;
+  REQUIRE(x && w && y, "null pointer argument");
+  REQUIRE(aligned16(x) && aligned16(w), "x and w must be 16-byte aligned");
+  qsa::ProjectArgs a{x, w, T, H, N, y, dev_status};
+  return cuda_status(qsa::launch_indexer_project(a, x_dt, w_dt, (cudaStream_t)stream), "qsa_indexer_project launch");
+}
+
+size_t qsa_compress_keys_workspace_size(int n_groups, int D_I) {
+  (void)n_groups; (void)D_I;
+  return 0;
+}
+
+qsa_status_t qsa_compress_keys(const float* k_tok, int tok_stride, int n_groups, const int32_t* g_req,
+                               const int32_t* g_id, const float* wphi, const float* bias, int D_I,
+                               void* k_idx_pages, qsa_dtype_t k_dt, int num_pages, const int32_t* page_table,
+                               int pt_rows, int pt_stride, uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(n_groups >= 0, "n_groups must be >= 0 (got %d)", n_groups);
+  SUPPORT(D_I == 32 || D_I == 64 || D_I == 128, "D_I must be 32, 64 or 128 (got %d)", D_I);
+  REQUIRE(tok_stride >= D_I, "tok_stride %d is smaller than D_I %d", tok_stride, D_I);
+  REQUIRE(k_dt == QSA_F32 || k_dt == QSA_BF16, "k_idx_pages dtype must be F32 or BF16");
+  REQUIRE(num_pages >= 1 && pt_rows >= 1 && pt_stride >= 1, "num_pages, pt_rows and pt_stride must be >= 1");
+  SUPPORT(n_groups <= (1 << 30), "n_groups = %d is too large", n_groups);
+  if (n_groups == 0) return QSA_OK;
+  REQUIRE(k_tok && g_id && wphi && k_idx_pages && page_table, "null pointer argument");
+  qsa::CompressArgs c{k_tok, tok_stride, n_groups, g_req, g_id, wphi, bias, D_I, k_idx_pages, num_pages,
+                      page_table, pt_rows, pt_stride, dev_status};
+  return cuda_status(qsa::launch_compress_keys(c, k_dt, (cudaStream_t)stream), "qsa_compress_keys launch");
 }
 
 qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* w_idx,

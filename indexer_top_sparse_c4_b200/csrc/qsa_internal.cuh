@@ -252,6 +252,21 @@ cudaError_t launch_sparse_attn_gather(const AttnArgs& a, float qk_scale_log2, fl
 cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
                                     int s, void* ws, cudaStream_t stream);
 
+// Indexer projection y[T, N] = x[T, H] . w[N, H]^T (indexer_write.cu): a GEMV
+// for few tokens, a tcgen05 GEMM for BF16 prefill chunks.
+struct ProjectArgs {
+  const void* x; const void* w; int T, H, N; float* y; uint32_t* status;
+};
+bool project_tc_supported(const ProjectArgs& a, qsa_dtype_t x_dt, qsa_dtype_t w_dt);
+cudaError_t launch_indexer_project(const ProjectArgs& a, qsa_dtype_t x_dt, qsa_dtype_t w_dt, cudaStream_t s);
+// C4 compressed-key write (indexer_write.cu).
+struct CompressArgs {
+  const float* k_tok; int tok_stride; int n; const int32_t* g_req; const int32_t* g_id;
+  const float* wphi; const float* bias; int D_I; void* k_idx_pages; int num_pages;
+  const int32_t* page_table; int pt_rows, pt_stride; uint32_t* status;
+};
+cudaError_t launch_compress_keys(const CompressArgs& c, qsa_dtype_t k_dt, cudaStream_t s);
+
 // Sets the message qsa_last_error_string() returns on this thread.
 void set_last_error(const char* msg);
 // The host-side argument checks of the attention calls (shapes, dtypes,

@@ -25,6 +25,8 @@ QSA_DEV_BAD_REQUEST, QSA_DEV_TIMEOUT = 16, 32
 QSA_PREFIX_HIST_BINS = 4096
 
 ENTRY_POINTS = (
+    "qsa_indexer_project_workspace_size", "qsa_indexer_project", "qsa_compress_keys_workspace_size",
+    "qsa_compress_keys",
     "qsa_index_scores_workspace_size", "qsa_index_scores", "qsa_topk_groups_workspace_size",
     "qsa_topk_groups", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
@@ -52,6 +54,14 @@ def lib() -> ctypes.CDLL:
                            "`python -m indexer_top_sparse_c4_b200.build` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     P, I, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.qsa_indexer_project_workspace_size.argtypes = [I, I, I]
+    L.qsa_indexer_project_workspace_size.restype = U
+    L.qsa_indexer_project.argtypes = [P, I, P, I, I, I, I, P, P, P]
+    L.qsa_indexer_project.restype = I
+    L.qsa_compress_keys_workspace_size.argtypes = [I, I]
+    L.qsa_compress_keys_workspace_size.restype = U
+    L.qsa_compress_keys.argtypes = [P, I, I, P, P, P, P, I, P, I, I, P, I, I, P, P]
+    L.qsa_compress_keys.restype = I
     L.qsa_index_scores_workspace_size.argtypes = [I, I, I, I]
     L.qsa_index_scores_workspace_size.restype = U
     L.qsa_expand_select_workspace_size.argtypes = [I, I, I]
@@ -131,6 +141,35 @@ def qsa_index_scores(q_idx, w_idx, k_idx_pages, page_table, q_pos, scores, q_req
         T, H_I, D_I, _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(dev_status),
         _stream(stream)))
     return scores
+
+
+def qsa_indexer_project(x, w, y, dev_status=None, stream=None):
+    """y [T, N] float32 = x [T, H] . w [N, H]^T (x and w float32 or bfloat16)."""
+    T, H = x.shape
+    N, H2 = w.shape
+    if H2 != H or tuple(y.shape) != (T, N) or y.dtype != torch.float32:
+        raise ValueError("shapes: x [T, H], w [N, H], y [T, N] float32")
+    _check(lib().qsa_indexer_project(_ptr(x), _dt(x), _ptr(w), _dt(w), T, H, N, _ptr(y), _ptr(dev_status),
+                                     _stream(stream)))
+    return y
+
+
+def qsa_compress_keys(k_tok, g_id, wphi, k_idx_pages, page_table, g_req=None, bias=None, dev_status=None,
+                      stream=None):
+    """The C4 compressed-key write.  k_tok: float32 [4 * n, D_I] token keys,
+    four consecutive rows per completed group; its rows may be strided (a
+    column slice of qsa_indexer_project's output) but each row contiguous."""
+    if k_tok.dtype != torch.float32 or k_tok.dim() != 2 or k_tok.stride(1) != 1:
+        raise ValueError("k_tok must be float32 [4 * n, D_I] with contiguous rows")
+    rows, D_I = k_tok.shape
+    n = g_id.numel()
+    if rows != 4 * n:
+        raise ValueError("k_tok must hold four token rows per group")
+    _check(lib().qsa_compress_keys(
+        ctypes.c_void_p(k_tok.data_ptr()), k_tok.stride(0), n, _ptr(g_req), _ptr(g_id), _ptr(wphi), _ptr(bias),
+        D_I, _ptr(k_idx_pages), _dt(k_idx_pages), k_idx_pages.shape[0], _ptr(page_table), page_table.shape[0],
+        page_table.shape[1], _ptr(dev_status), _stream(stream)))
+    return k_idx_pages
 
 
 def qsa_index_scores_workspace_size(T, H_I, D_I, score_stride) -> int:

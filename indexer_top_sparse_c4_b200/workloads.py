@@ -218,6 +218,30 @@ def make(name: str, *, B: int, ctx: int, Hq: int, Hkv: int, D: int, H_I: int, D_
                     capture_pos=capture_pos, dist=dist, seed=seed)
 
 
+def indexer_weights(hidden: int, H_I: int = 4, D_I: int = 128, seed: int = 0, device="cpu",
+                    dtype: str = "bf16"):
+    """Synthetic, seeded weights of the indexer's projection and of the C4
+    compression (there is no checkpoint): w [H_I*D_I + H_I + D_I, hidden]
+    stacking W_q, W_w, W_k with N(0, 1/hidden) entries (so projected values
+    are about N(0, 1)), wphi [D_I, 4*D_I] = mean pooling [I/4 x 4] plus
+    N(0, 0.02^2) entries, and bias [D_I] ~ N(0, 0.01^2).  Returns
+    (w, wphi, bias); w in the given storage type, the others float32."""
+    g = _gen(seed, device)
+    N = H_I * D_I + H_I + D_I
+    w = _randn((N, hidden), g, device) / float(hidden) ** 0.5
+    eye = torch.eye(D_I, device=device, dtype=torch.float32)
+    wphi = torch.cat([eye / GROUP_TOKENS] * GROUP_TOKENS, dim=1) + 0.02 * _randn((D_I, GROUP_TOKENS * D_I), g, device)
+    bias = 0.01 * _randn((D_I,), g, device)
+    w, _ = _store(w, dtype)
+    return w, wphi.contiguous(), bias.contiguous()
+
+
+def hidden_states(T: int, hidden: int, seed: int = 0, device="cpu", dtype: str = "bf16") -> torch.Tensor:
+    """Synthetic hidden states x [T, hidden] ~ N(0, 1) in the given storage type."""
+    x, _ = _store(_randn((T, hidden), _gen(seed, device), device), dtype)
+    return x
+
+
 # ---- the named workloads --------------------------------------------------------
 
 def tiny(device="cpu", seed=0, **kw) -> Workload:

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 5
+    assert L.qsa_abi_version() == 6
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -181,3 +181,23 @@ def test_device_status_query_checks_its_pointer(L):
     assert L.qsa_get_device_status(ctypes.c_void_p(0x2002), ctypes.byref(bits), 1, NULL) == 1
     assert "aligned" in _err(L)
     assert bits.value == 7
+
+
+def test_indexer_write_validation(L):
+    ok = ctypes.c_void_p(0x2000)
+    # (x, x_dt, w, w_dt, T, H, N, y, status, stream)
+    assert L.qsa_indexer_project(ok, 1, ok, 1, 8, 5120, 0, ok, NULL, NULL) == 1
+    assert L.qsa_indexer_project(ok, 2, ok, 1, 8, 5120, 644, ok, NULL, NULL) == 1 and "dtype" in _err(L)
+    assert L.qsa_indexer_project(ok, 1, ok, 1, 8, 5121, 644, ok, NULL, NULL) == 2
+    assert L.qsa_indexer_project(NULL, 1, ok, 1, 8, 5120, 644, ok, NULL, NULL) == 1 and "null" in _err(L)
+    assert L.qsa_indexer_project(ctypes.c_void_p(0x2004), 1, ok, 1, 8, 5120, 644, ok, NULL, NULL) == 1
+    assert L.qsa_indexer_project(NULL, 1, NULL, 1, 0, 5120, 644, NULL, NULL, NULL) == 0
+    assert L.qsa_indexer_project_workspace_size(8192, 5120, 644) == 0
+    # (k_tok, tok_stride, n, g_req, g_id, wphi, bias, D_I, pages, k_dt, num_pages, pt, pt_rows, pt_stride, st, s)
+    assert L.qsa_compress_keys(ok, 128, 4, NULL, ok, ok, NULL, 96, ok, 0, 4, ok, 1, 4, NULL, NULL) == 2
+    assert L.qsa_compress_keys(ok, 64, 4, NULL, ok, ok, NULL, 128, ok, 0, 4, ok, 1, 4, NULL, NULL) == 1
+    assert "tok_stride" in _err(L)
+    assert L.qsa_compress_keys(ok, 128, 4, NULL, ok, ok, NULL, 128, ok, 2, 4, ok, 1, 4, NULL, NULL) == 1
+    assert L.qsa_compress_keys(ok, 128, 4, NULL, NULL, ok, NULL, 128, ok, 0, 4, ok, 1, 4, NULL, NULL) == 1
+    assert L.qsa_compress_keys(NULL, 128, 0, NULL, NULL, NULL, NULL, 128, NULL, 0, 4, NULL, 1, 4, NULL, NULL) == 0
+    assert L.qsa_compress_keys_workspace_size(2048, 128) == 0
