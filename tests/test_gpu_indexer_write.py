@@ -93,13 +93,15 @@ def _check_compress(q, oracle, k_tok, g_id, g_req, pt, num_pages, dt, seed=0):
     for r, g in zip(req_h, gid_h):
         written[pt_h[r, g // 16], g % 16] = True
     assert np.array_equal(got[~written], want[~written])
-    # written rows: within the dot-product bound (plus one BF16 step for BF16 storage)
+    # written rows: within the dot-product bound; with BF16 storage both sides
+    # round values that differ within that bound, so they may land on
+    # neighbouring BF16 values: one step, at most |v| * 2^-7
     wphi_h, b_h = host(wphi).astype(np.float64), host(bias).astype(np.float64)
     for i, (r, g) in enumerate(zip(req_h, gid_h)):
         p, row = pt_h[r, g // 16], g % 16
         scale = np.abs(wphi_h) @ np.abs(kt[i].reshape(-1).astype(np.float64)) + np.abs(b_h)
         gv, wv = values_f64(got[p, row]), values_f64(want[p, row])
-        tol = SCORE_REL * scale + (np.abs(wv) * 2.0 ** -8 if dt == "bf16" else 0.0)
+        tol = SCORE_REL * scale + (np.abs(wv) * 2.0 ** -7 if dt == "bf16" else 0.0)
         assert np.all(np.abs(gv - wv) <= tol + 1e-30), (i, float(np.abs(gv - wv).max()))
     return pages
 
