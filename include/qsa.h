@@ -292,6 +292,60 @@ QSA_API qsa_status_t qsa_sparse_attn_decode_noalloc(
     int Hq, int Hkv, int D, float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
     uint32_t* dev_status, qsa_stream_t stream);
 
+/* Sequence-sharded decode (decode context parallelism; the Ascend article's
+ * context section names it for the QSA path).  R shards each hold a
+ * contiguous range of every request's pages -- shard r the groups
+ * [g_lo, g_hi), g_lo a multiple of 16 -- as a slice of the page table over
+ * the same (or its own) KV cache and compressed keys.  A decode step:
+ *   qsa_dcp_shard_positions  -> q_pos_local (per shard)
+ *   qsa_index_scores, qsa_topk_groups on the shard (q_pos_local, its slice)
+ *   qsa_dcp_candidates       -> (score, global group id) records [T, K]
+ *   all-gather of the records over the shards -> [R, T, K] (shard order)
+ *   qsa_dcp_merge_topk       -> the global selection sel [T, K], n_sel [T]
+ *   qsa_dcp_expand           -> the shard's token lists (shard-local ids)
+ *   qsa_sparse_attn_decode on the shard (F32 out, lse) -> partials
+ *   all-gather of the partials -> [R, T, Hq, D], [R, T, Hq]
+ *   qsa_dcp_merge_attn       -> out [T, Hq, D], lse [T, Hq]
+ * The selection is exactly the one unsharded stage 2 makes from the same
+ * scores (each of the global K best is among the K best of its shard), and
+ * the merged output is the attention over the same tokens. */
+/* q_pos_local[t] = 4 * clamp(q_pos[t] / 4 - g_lo, 0, g_hi - g_lo): the shard's
+ * candidate count as a query position, for stages 1 and 2 on the slice. */
+QSA_API qsa_status_t qsa_dcp_shard_positions(const int32_t* q_pos, int T, int g_lo, int g_hi,
+                                             int32_t* q_pos_local, qsa_stream_t stream);
+/* The shard's selection sel/n_sel [T, K] (shard-local ids, ascending, from
+ * qsa_topk_groups on its scores [T, score_stride]) as records:
+ * cand_id = sel + g_lo, cand_score = that group's score; slots past n_sel
+ * get (-inf, -1).  A sel entry outside [0, score_stride) becomes (-inf, -1)
+ * and sets QSA_DEV_BAD_GROUP. */
+QSA_API qsa_status_t qsa_dcp_candidates(const float* scores, int score_stride, const int32_t* sel,
+                                        const int32_t* n_sel, int T, int K, int g_lo, float* cand_score,
+                                        int32_t* cand_id, uint32_t* dev_status, qsa_stream_t stream);
+/* The global top-K of the gathered records cand_score / cand_id [R, T, K]
+ * (shard r's block at r * T * K): n_sel[t] = min(K, real records of row t),
+ * sel[t] their ids ranked by (score descending, id ascending), written in
+ * ascending id order and padded with -1.  The output order relies on the
+ * records ascending by id in (shard, slot) order, which holds for records
+ * of shards with ascending group ranges.  R * K <= 16384. */
+QSA_API qsa_status_t qsa_dcp_merge_topk(const float* cand_score, const int32_t* cand_id, int R, int T, int K,
+                                        int32_t* sel, int32_t* n_sel, qsa_stream_t stream);
+/* The shard's part of the global selection sel/n_sel [T, K] (ascending global
+ * ids): tokens 4(g - g_lo) .. 4(g - g_lo) + 3 of every selected g in
+ * [g_lo, g_hi), then -- when the current block c = q_pos[t] / 4 lies in
+ * [g_lo, g_hi) -- its tokens 4(c - g_lo) .. q_pos[t] - 4 g_lo, as shard-local
+ * token ids, ascending, -1 padded to W; n_tok[t] the count.  A row wider than
+ * W is cut and sets QSA_DEV_ROW_RANGE. */
+QSA_API qsa_status_t qsa_dcp_expand(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos, int T,
+                                    int g_lo, int g_hi, int32_t* tok, int32_t* n_tok, int W,
+                                    uint32_t* dev_status, qsa_stream_t stream);
+/* LSE merge of R partial attentions: o_parts [R, T, Hq, D] (F32, each
+ * normalised over its shard's tokens) and lse_parts [R, T, Hq] (natural log,
+ * -inf for a shard without tokens): out = sum_r exp(lse_r - LSE) o_r with
+ * LSE = log sum_r exp(lse_r); rows where every shard is empty give 0 and
+ * -inf.  out_dt F32 or BF16; lse may be NULL. */
+QSA_API qsa_status_t qsa_dcp_merge_attn(const float* o_parts, const float* lse_parts, int R, int T, int Hq, int D,
+                                        void* out, qsa_dtype_t out_dt, float* lse, qsa_stream_t stream);
+
 /* Device status query (the boundary's error channel for data the kernels
  * check on the device; see "Conventions" above).  Waits for `stream` to finish
  * the work queued so far, reads the caller's status word dev_status and
@@ -318,7 +372,7 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand; 5: the
  * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
  * and a workspace query for every stage; 6: qsa_indexer_project and
- * qsa_compress_keys). */
+ * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -36,6 +36,7 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
   } while (0)
 
 constexpr int kMaxGridY = 65535;
+constexpr int kPageGroupsAbi = 16;   // groups per 64-token page
 
 qsa_status_t check_attn(const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages,
                         qsa_dtype_t kv_dt, int num_pages, const int32_t* page_table, int pt_rows,
@@ -96,7 +97,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 6; }
+int qsa_abi_version(void) { return 7; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -206,6 +207,65 @@ qsa_status_t qsa_index_scores(const void* q_idx, qsa_dtype_t q_dt, const float* 
                             ? qsa::launch_index_scores_tc(a, (cudaStream_t)stream)
                             : qsa::launch_index_scores(a, (cudaStream_t)stream);
   return cuda_status(e, "qsa_index_scores launch");
+}
+
+qsa_status_t qsa_dcp_shard_positions(const int32_t* q_pos, int T, int g_lo, int g_hi, int32_t* q_pos_local,
+                                     qsa_stream_t stream) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  REQUIRE(g_lo >= 0 && g_hi >= g_lo, "need 0 <= g_lo <= g_hi (got %d, %d)", g_lo, g_hi);
+  REQUIRE(g_lo % kPageGroupsAbi == 0, "shard boundaries must fall on pages: g_lo %% 16 == 0 (got %d)", g_lo);
+  if (T == 0) return QSA_OK;
+  REQUIRE(q_pos && q_pos_local, "null pointer argument");
+  return cuda_status(qsa::launch_dcp_positions(q_pos, T, g_lo, g_hi, q_pos_local, (cudaStream_t)stream),
+                     "qsa_dcp_shard_positions launch");
+}
+
+qsa_status_t qsa_dcp_candidates(const float* scores, int score_stride, const int32_t* sel, const int32_t* n_sel,
+                                int T, int K, int g_lo, float* cand_score, int32_t* cand_id, uint32_t* dev_status,
+                                qsa_stream_t stream) {
+  REQUIRE(T >= 0 && K >= 1 && score_stride >= 1 && g_lo >= 0, "need T >= 0, K >= 1, score_stride >= 1, g_lo >= 0");
+  if (T == 0) return QSA_OK;
+  REQUIRE(scores && sel && n_sel && cand_score && cand_id, "null pointer argument");
+  return cuda_status(qsa::launch_dcp_candidates(scores, score_stride, sel, n_sel, T, K, g_lo, cand_score, cand_id,
+                                                dev_status, (cudaStream_t)stream),
+                     "qsa_dcp_candidates launch");
+}
+
+qsa_status_t qsa_dcp_merge_topk(const float* cand_score, const int32_t* cand_id, int R, int T, int K, int32_t* sel,
+                                int32_t* n_sel, qsa_stream_t stream) {
+  REQUIRE(T >= 0 && K >= 1 && R >= 1, "need T >= 0, K >= 1, R >= 1 (got %d, %d, %d)", T, K, R);
+  SUPPORT((long long)R * K <= qsa::dcp_merge_max_candidates(), "R * K = %lld exceeds the %d candidates a row may merge",
+          (long long)R * K, qsa::dcp_merge_max_candidates());
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  if (T == 0) return QSA_OK;
+  REQUIRE(cand_score && cand_id && sel && n_sel, "null pointer argument");
+  return cuda_status(qsa::launch_dcp_merge_topk(cand_score, cand_id, R, T, K, sel, n_sel, (cudaStream_t)stream),
+                     "qsa_dcp_merge_topk launch");
+}
+
+qsa_status_t qsa_dcp_expand(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos, int T, int g_lo,
+                            int g_hi, int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
+                            qsa_stream_t stream) {
+  REQUIRE(T >= 0 && K >= 1 && W >= 1, "need T >= 0, K >= 1, W >= 1");
+  REQUIRE(g_lo >= 0 && g_hi >= g_lo, "need 0 <= g_lo <= g_hi (got %d, %d)", g_lo, g_hi);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  if (T == 0) return QSA_OK;
+  REQUIRE(sel && n_sel && q_pos && tok && n_tok, "null pointer argument");
+  return cuda_status(qsa::launch_dcp_expand(sel, n_sel, K, q_pos, T, g_lo, g_hi, tok, n_tok, W, dev_status,
+                                            (cudaStream_t)stream),
+                     "qsa_dcp_expand launch");
+}
+
+qsa_status_t qsa_dcp_merge_attn(const float* o_parts, const float* lse_parts, int R, int T, int Hq, int D, void* out,
+                                qsa_dtype_t out_dt, float* lse, qsa_stream_t stream) {
+  REQUIRE(T >= 0 && R >= 1 && Hq >= 1 && D >= 1, "need T >= 0, R, Hq, D >= 1");
+  REQUIRE(out_dt == QSA_F32 || out_dt == QSA_BF16, "out dtype must be F32 or BF16");
+  SUPPORT((long long)T * Hq <= 0x7fffffffLL, "T * Hq too large");
+  if (T == 0) return QSA_OK;
+  REQUIRE(o_parts && lse_parts && out, "null pointer argument");
+  return cuda_status(qsa::launch_dcp_merge_attn(o_parts, lse_parts, R, T, Hq, D, out, out_dt, lse,
+                                                (cudaStream_t)stream),
+                     "qsa_dcp_merge_attn launch");
 }
 
 size_t qsa_topk_groups_workspace_size(int T, int K, int score_stride) {

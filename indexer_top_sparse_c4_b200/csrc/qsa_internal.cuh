@@ -267,6 +267,20 @@ struct CompressArgs {
 };
 cudaError_t launch_compress_keys(const CompressArgs& c, qsa_dtype_t k_dt, cudaStream_t s);
 
+// Sequence-sharded decode (dcp.cu).
+cudaError_t launch_dcp_positions(const int32_t* q_pos, int T, int g_lo, int g_hi, int32_t* q_pos_local,
+                                 cudaStream_t s);
+cudaError_t launch_dcp_candidates(const float* scores, int score_stride, const int32_t* sel, const int32_t* n_sel,
+                                  int T, int K, int g_lo, float* cand_score, int32_t* cand_id, uint32_t* status,
+                                  cudaStream_t s);
+int dcp_merge_max_candidates();
+cudaError_t launch_dcp_merge_topk(const float* cand_score, const int32_t* cand_id, int R, int T, int K, int32_t* sel,
+                                  int32_t* n_sel, cudaStream_t s);
+cudaError_t launch_dcp_expand(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos, int T, int g_lo,
+                              int g_hi, int32_t* tok, int32_t* n_tok, int W, uint32_t* status, cudaStream_t s);
+cudaError_t launch_dcp_merge_attn(const float* o_parts, const float* lse_parts, int R, int T, int Hq, int D,
+                                  void* out, qsa_dtype_t out_dt, float* lse, cudaStream_t s);
+
 // Sets the message qsa_last_error_string() returns on this thread.
 void set_last_error(const char* msg);
 // The host-side argument checks of the attention calls (shapes, dtypes,

@@ -31,6 +31,8 @@ ENTRY_POINTS = (
     "qsa_topk_groups", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
     "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
+    "qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
+    "qsa_dcp_merge_attn",
     "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
 )
 
@@ -62,6 +64,14 @@ def lib() -> ctypes.CDLL:
     L.qsa_compress_keys_workspace_size.restype = U
     L.qsa_compress_keys.argtypes = [P, I, I, P, P, P, P, I, P, I, I, P, I, I, P, P]
     L.qsa_compress_keys.restype = I
+    L.qsa_dcp_shard_positions.argtypes = [P, I, I, I, P, P]
+    L.qsa_dcp_candidates.argtypes = [P, I, P, P, I, I, I, P, P, P, P]
+    L.qsa_dcp_merge_topk.argtypes = [P, P, I, I, I, P, P, P]
+    L.qsa_dcp_expand.argtypes = [P, P, I, P, I, I, I, P, P, I, P, P]
+    L.qsa_dcp_merge_attn.argtypes = [P, P, I, I, I, I, P, I, P, P]
+    for name in ("qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
+                 "qsa_dcp_merge_attn"):
+        getattr(L, name).restype = I
     L.qsa_index_scores_workspace_size.argtypes = [I, I, I, I]
     L.qsa_index_scores_workspace_size.restype = U
     L.qsa_expand_select_workspace_size.argtypes = [I, I, I]
@@ -293,4 +303,42 @@ def qsa_sparse_attn_decode_noalloc(q, k_pages, v_pages, page_table, tok, n_tok, 
     args = _attn_args(q, k_pages, v_pages, page_table, tok, n_tok, out, k_scale, v_scale, q_req,
                       sm_scale, lse)
     _check(fn(*args, _ptr(dev_status), _stream(stream)))
+    return out
+
+
+# ---- sequence-sharded decode ---------------------------------------------------------
+
+def qsa_dcp_shard_positions(q_pos, g_lo, g_hi, q_pos_local, stream=None):
+    _check(lib().qsa_dcp_shard_positions(_ptr(q_pos), q_pos.numel(), g_lo, g_hi, _ptr(q_pos_local),
+                                         _stream(stream)))
+    return q_pos_local
+
+
+def qsa_dcp_candidates(scores, sel, n_sel, g_lo, cand_score, cand_id, dev_status=None, stream=None):
+    T, K = sel.shape
+    _check(lib().qsa_dcp_candidates(_ptr(scores), scores.shape[1], _ptr(sel), _ptr(n_sel), T, K, g_lo,
+                                    _ptr(cand_score), _ptr(cand_id), _ptr(dev_status), _stream(stream)))
+    return cand_score, cand_id
+
+
+def qsa_dcp_merge_topk(cand_score, cand_id, sel, n_sel, stream=None):
+    """cand_score / cand_id [R, T, K] -> sel [T, K], n_sel [T]."""
+    R, T, K = cand_id.shape
+    _check(lib().qsa_dcp_merge_topk(_ptr(cand_score), _ptr(cand_id), R, T, K, _ptr(sel), _ptr(n_sel),
+                                    _stream(stream)))
+    return sel, n_sel
+
+
+def qsa_dcp_expand(sel, n_sel, q_pos, g_lo, g_hi, tok, n_tok, dev_status=None, stream=None):
+    T, K = sel.shape
+    _check(lib().qsa_dcp_expand(_ptr(sel), _ptr(n_sel), K, _ptr(q_pos), T, g_lo, g_hi, _ptr(tok), _ptr(n_tok),
+                                tok.shape[1], _ptr(dev_status), _stream(stream)))
+    return tok, n_tok
+
+
+def qsa_dcp_merge_attn(o_parts, lse_parts, out, lse=None, stream=None):
+    """o_parts [R, T, Hq, D] float32, lse_parts [R, T, Hq] -> out [T, Hq, D], lse [T, Hq]."""
+    R, T, Hq, D = o_parts.shape
+    _check(lib().qsa_dcp_merge_attn(_ptr(o_parts), _ptr(lse_parts), R, T, Hq, D, _ptr(out), _dt(out), _ptr(lse),
+                                    _stream(stream)))
     return out
