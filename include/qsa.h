@@ -191,6 +191,24 @@ QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint
                              void* workspace, size_t workspace_bytes, uint32_t* dev_status,
                              qsa_stream_t stream);
 
+/* Stage 2 as a guess-verify-refine Top-K with hint-free self-sampling
+ * (TensorRT-LLM "QSASparseAttentionConfig", enable_heuristic_topk: the GVR
+ * Top-K, for group budgets of 512, 1,024 and 2,048, falling back to the exact
+ * radix Top-K otherwise).  Same inputs, outputs and result as
+ * qsa_topk_groups: the exact top-min(K, c) of every row, ties to the lower
+ * group id, ascending, -1 padded.  Per row it guesses a threshold from a
+ * strided sample of the row's own scores, verifies by counting the scores
+ * that reach it (re-guessing from the sample when the count is too small or
+ * too large), and refines with an exact select among the gathered
+ * candidates; a row whose guesses fail takes a radix select over the whole
+ * row.  path (optional, [T] int32) receives per row: 0 dense (c <= K), 1 the
+ * first guess verified, 2 a later guess verified, 3 the whole-row select.
+ * For K outside {512, 1024, 2048} the call runs qsa_topk_groups instead (a
+ * message on stderr the first time) and leaves path unwritten. */
+QSA_API qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,
+                                         int32_t* sel, int32_t* n_sel, int32_t* path, uint32_t* dev_status,
+                                         qsa_stream_t stream);
+
 /* Stage 3 -- expansion of the kept groups to token ids ("QSA in brief": the
  * budget plus the current block; TensorRT-LLM get_indices_block_size: the
  * selections address single tokens; the MTP index-sharing field).
@@ -372,7 +390,8 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * argument of qsa_index_scores, qsa_topk_groups and qsa_topk_expand; 5: the
  * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
  * and a workspace query for every stage; 6: qsa_indexer_project and
- * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*). */
+ * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*; 8:
+ * qsa_topk_groups_gvr). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -97,7 +97,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 7; }
+int qsa_abi_version(void) { return 8; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -290,6 +290,30 @@ qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint32_t* pr
   qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
   a.hist = prefix_hist;
   return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups launch");
+}
+
+qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,
+                                 int32_t* sel, int32_t* n_sel, int32_t* path, uint32_t* dev_status,
+                                 qsa_stream_t stream) {
+  REQUIRE(T >= 0, "T must be >= 0 (got %d)", T);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
+  REQUIRE(score_stride >= 1, "score_stride must be >= 1");
+  if (!qsa::topk_gvr_budget(K)) {
+    // the pages' prerequisite for the self-sampling engine: the exact radix
+    // Top-K runs instead, with a warning the first time
+    static bool warned = false;
+    if (!warned) {
+      warned = true;
+      fprintf(stderr, "qsa_topk_groups_gvr: budget K = %d is not 512, 1024 or 2048; using the exact radix Top-K\n",
+              K);
+    }
+    return qsa_topk_groups(scores, score_stride, nullptr, q_pos, T, K, sel, n_sel, nullptr, 0, dev_status, stream);
+  }
+  if (T == 0) return QSA_OK;
+  REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
+  return cuda_status(qsa::launch_topk_gvr(scores, score_stride, q_pos, T, K, sel, n_sel, path, (cudaStream_t)stream),
+                     "qsa_topk_groups_gvr launch");
 }
 
 qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos,

@@ -267,6 +267,11 @@ struct CompressArgs {
 };
 cudaError_t launch_compress_keys(const CompressArgs& c, qsa_dtype_t k_dt, cudaStream_t s);
 
+// Guess-verify-refine Top-K with self-sampling (topk_gvr.cu).
+bool topk_gvr_budget(int K);
+cudaError_t launch_topk_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K, int32_t* sel,
+                            int32_t* n_sel, int32_t* path, cudaStream_t s);
+
 // Sequence-sharded decode (dcp.cu).
 cudaError_t launch_dcp_positions(const int32_t* q_pos, int T, int g_lo, int g_hi, int32_t* q_pos_local,
                                  cudaStream_t s);

@@ -28,7 +28,7 @@ ENTRY_POINTS = (
     "qsa_indexer_project_workspace_size", "qsa_indexer_project", "qsa_compress_keys_workspace_size",
     "qsa_compress_keys",
     "qsa_index_scores_workspace_size", "qsa_index_scores", "qsa_topk_groups_workspace_size",
-    "qsa_topk_groups", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
+    "qsa_topk_groups", "qsa_topk_groups_gvr", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
     "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
     "qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
     L.qsa_compress_keys_workspace_size.restype = U
     L.qsa_compress_keys.argtypes = [P, I, I, P, P, P, P, I, P, I, I, P, I, I, P, P]
     L.qsa_compress_keys.restype = I
+    L.qsa_topk_groups_gvr.argtypes = [P, I, P, I, I, P, P, P, P, P]
+    L.qsa_topk_groups_gvr.restype = I
     L.qsa_dcp_shard_positions.argtypes = [P, I, I, I, P, P]
     L.qsa_dcp_candidates.argtypes = [P, I, P, P, I, I, I, P, P, P, P]
     L.qsa_dcp_merge_topk.argtypes = [P, P, I, I, I, P, P, P]
@@ -219,6 +221,15 @@ def qsa_topk_groups(scores, q_pos, K, sel, n_sel, workspace=None, dev_status=Non
     _check(lib().qsa_topk_groups(
         _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel),
         _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
+    return sel, n_sel
+
+
+def qsa_topk_groups_gvr(scores, q_pos, K, sel, n_sel, path=None, dev_status=None, stream=None):
+    """The guess-verify-refine Top-K (same result as qsa_topk_groups);
+    path: optional int32 [T] receiving how each row was selected."""
+    T = scores.shape[0]
+    _check(lib().qsa_topk_groups_gvr(_ptr(scores), scores.shape[1], _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel),
+                                     _ptr(path), _ptr(dev_status), _stream(stream)))
     return sel, n_sel
 
 

@@ -1,0 +1,105 @@
+"""The guess-verify-refine Top-K (self-sampling): the same selection as the
+exact radix Top-K and the oracle, bit for bit, on the GPU's own scores, for
+every budget it serves and every score distribution; the path record shows
+that the self-sampled guess is what selects on ordinary rows, and that rows
+where guessing cannot work (thousands of equal scores) take the whole-row
+select."""
+import numpy as np
+import pytest
+import torch
+
+from indexer_top_sparse_c4_b200 import workloads as wl
+from indexer_top_sparse_c4_b200.pipeline import QSAStep
+from parity_utils import host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def q():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from indexer_top_sparse_c4_b200 import build, qsa
+    build.build()
+    return qsa
+
+
+def _gvr(q, scores, q_pos, K):
+    T = scores.shape[0]
+    sel = torch.full((T, K), 7, dtype=torch.int32, device="cuda")
+    n_sel = torch.full((T,), 7, dtype=torch.int32, device="cuda")
+    path = torch.full((T,), -1, dtype=torch.int32, device="cuda")
+    q.qsa_topk_groups_gvr(scores, q_pos, K, sel, n_sel, path=path)
+    torch.cuda.synchronize()
+    return sel, n_sel, path
+
+
+def _radix(q, scores, q_pos, K):
+    T = scores.shape[0]
+    sel = torch.empty((T, K), dtype=torch.int32, device="cuda")
+    n_sel = torch.empty((T,), dtype=torch.int32, device="cuda")
+    q.qsa_topk_groups(scores, q_pos, K, sel, n_sel)
+    torch.cuda.synchronize()
+    return sel, n_sel
+
+
+@pytest.mark.parametrize("K", [512, 1024, 2048])
+@pytest.mark.parametrize("dist", ["peaked", "normal", "ties"])
+def test_gvr_equals_radix_and_oracle_on_decode_rows(q, oracle, K, dist):
+    w = wl.b8_262k(K=K, device="cuda", dist=dist, B=4, ctx=65536 if dist == "ties" else 262144)
+    st = QSAStep(w, prefix_hist=False)
+    st.index_scores()
+    sel, n_sel, path = _gvr(q, st.scores, w.q_pos, K)
+    rs, rn = _radix(q, st.scores, w.q_pos, K)
+    assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
+    ref, nref = oracle.topk_groups(host(st.scores), host(w.q_pos), K)
+    assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref)
+    p = host(path)
+    if dist == "ties":   # 16 score levels: the guess may land on a crowded level
+        assert set(p.tolist()) <= {1, 2, 3}
+    else:
+        assert np.all(p == 1), p                     # the first self-sampled guess verifies
+
+
+def test_gvr_rows_of_every_length(q, oracle):
+    """Prefill-like rows: dense rows (c <= K), rows just above K, long rows,
+    an odd score stride; all against the radix Top-K and the oracle."""
+    T, ctx, K = 300, 16384, 512
+    pos = np.sort(np.random.default_rng(3).integers(4, ctx, T)).astype(np.int32)
+    pos[:4] = [5, 2047, 2051, 2052]
+    w = wl.make("rows", B=1, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=K, kv_dtype="bf16", q_dtype="bf16",
+                seed=4, device="cuda", q_pos=pos, q_req=np.zeros(T, np.int32))
+    st = QSAStep(w, score_stride=ctx // 4 + 1)
+    st.index_scores()
+    sel, n_sel, path = _gvr(q, st.scores, w.q_pos, K)
+    rs, rn = _radix(q, st.scores, w.q_pos, K)
+    assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
+    ref, nref = oracle.topk_groups(host(st.scores), host(w.q_pos), K)
+    assert np.array_equal(host(sel), ref)
+    p = host(path)
+    c = pos // 4
+    assert np.all(p[c <= K] == 0) and np.all(p[c > K] >= 1)
+
+
+def test_gvr_falls_back_on_equal_scores(q, oracle):
+    """Every candidate with the same score: no threshold can split them, the
+    row takes the whole-row select, and the lowest ids win."""
+    T, c, K = 2, 65535, 1024
+    scores = torch.zeros((T, c + 1), dtype=torch.float32, device="cuda")
+    scores[1, ::7] = -0.0                       # -0 ranks equal to +0
+    q_pos = torch.full((T,), 4 * c, dtype=torch.int32, device="cuda")
+    sel, n_sel, path = _gvr(q, scores, q_pos, K)
+    assert host(path).tolist() == [3, 3]
+    assert np.array_equal(host(sel), np.tile(np.arange(K, dtype=np.int32), (T, 1)))
+    ref, _ = oracle.topk_groups(host(scores), host(q_pos), K)
+    assert np.array_equal(host(sel), ref)
+
+
+def test_gvr_other_budgets_use_the_radix_top_k(q):
+    w = wl.b1_16k(device="cuda", K=300)
+    st = QSAStep(w)
+    st.index_scores()
+    sel, n_sel, path = _gvr(q, st.scores, w.q_pos, 300)
+    rs, rn = _radix(q, st.scores, w.q_pos, 300)
+    assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
+    assert host(path).tolist() == [-1]          # untouched: the radix Top-K ran
