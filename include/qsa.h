@@ -238,6 +238,20 @@ QSA_API qsa_status_t qsa_topk_expand(const float* scores, int score_stride, uint
                              int32_t* tok, int32_t* n_tok, int W, uint32_t* dev_status,
                              qsa_stream_t stream);
 
+/* The sequence-length threshold separating dense and QSA attention
+ * (TensorRT-LLM "QSASparseAttentionConfig", seq_len_threshold): `requested`
+ * tokens, or the token budget 4*K when requested <= 0; a value below 4*K is
+ * raised to 4*K, as it cannot reduce attention work.  Pure host function. */
+QSA_API int qsa_seq_len_threshold(int requested, int K);
+/* Dense rows of the threshold: every query whose sequence q_pos[t] + 1 is at
+ * most `threshold` tokens gets the token list 0 .. q_pos[t] (n_tok =
+ * q_pos[t] + 1, -1 padded to W), i.e. dense causal attention; the other rows
+ * of tok / n_tok are left as they are (the QSA selection of stage 3).  A
+ * dense row longer than W is cut and sets QSA_DEV_ROW_RANGE.  threshold <= 0:
+ * nothing is written. */
+QSA_API qsa_status_t qsa_dense_select(const int32_t* q_pos, int T, int threshold, int32_t* tok, int32_t* n_tok,
+                                      int W, uint32_t* dev_status, qsa_stream_t stream);
+
 /* Stage 4 -- GQA attention over the selected tokens ("QSA in brief": only the
  * selected entries are read; the Ascend article: rows with nothing to attend
  * give exact zeros, the D-based scale is the default).
@@ -391,7 +405,7 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
  * and a workspace query for every stage; 6: qsa_indexer_project and
  * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*; 8:
- * qsa_topk_groups_gvr). */
+ * qsa_topk_groups_gvr; 9: qsa_seq_len_threshold and qsa_dense_select). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

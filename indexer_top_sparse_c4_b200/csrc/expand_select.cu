@@ -46,7 +46,34 @@ __global__ void __launch_bounds__(kThreads) expand_kernel(ExpandArgs a) {
   }
 }
 
+// Dense rows of the sequence-length threshold ("QSASparseAttentionConfig",
+// seq_len_threshold): a query whose sequence (p + 1 tokens) is at most the
+// threshold attends to every token 0 .. p; other rows are left as they are.
+__global__ void __launch_bounds__(kThreads) dense_select_kernel(const int32_t* q_pos, int threshold, int32_t* tok,
+                                                                int32_t* n_tok, int W, uint32_t* status) {
+  pdl_wait();
+  const int t = blockIdx.y;
+  const int p = q_pos[t];
+  const int L = p + 1;
+  if (p < 0 || L > threshold) return;   // (whole CTA: the row is not dense)
+  int32_t* row = tok + (size_t)t * W;
+  for (int i = blockIdx.x * kThreads + threadIdx.x; i < W; i += gridDim.x * kThreads) row[i] = i < L ? i : -1;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    n_tok[t] = L < W ? L : W;
+    if (L > W) flag(status, QSA_DEV_ROW_RANGE);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_dense_select(const int32_t* q_pos, int T, int threshold, int32_t* tok, int32_t* n_tok, int W,
+                                uint32_t* status, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  int bx = (W + kThreads - 1) / kThreads;
+  if (bx > 64) bx = 64;
+  return launch_k(dense_select_kernel, dim3(bx, T), dim3(kThreads), 0, s, 1, q_pos, threshold, tok, n_tok, W,
+                  status);
+}
 
 cudaError_t launch_expand_select(const ExpandArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;

@@ -97,7 +97,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 8; }
+int qsa_abi_version(void) { return 9; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -327,6 +327,23 @@ qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, 
   REQUIRE(sel && n_sel && q_pos && tok && n_tok, "null pointer argument");
   qsa::ExpandArgs a{sel, n_sel, K, q_pos, capture_pos, T, tok, n_tok, W, dev_status};
   return cuda_status(qsa::launch_expand_select(a, (cudaStream_t)stream), "qsa_expand_select launch");
+}
+
+int qsa_seq_len_threshold(int requested, int K) {
+  const long long budget = 4ll * (K > 0 ? K : 0);   // the budget in tokens
+  const long long want = requested > 0 ? requested : budget;
+  const long long thr = want > budget ? want : budget;
+  return thr > 0x7fffffffLL ? 0x7fffffff : (int)thr;
+}
+
+qsa_status_t qsa_dense_select(const int32_t* q_pos, int T, int threshold, int32_t* tok, int32_t* n_tok, int W,
+                              uint32_t* dev_status, qsa_stream_t stream) {
+  REQUIRE(T >= 0 && W >= 1, "need T >= 0 and W >= 1 (got %d, %d)", T, W);
+  SUPPORT(T <= kMaxGridY, "T = %d exceeds %d query tokens per call", T, kMaxGridY);
+  if (T == 0 || threshold <= 0) return QSA_OK;
+  REQUIRE(q_pos && tok && n_tok, "null pointer argument");
+  return cuda_status(qsa::launch_dense_select(q_pos, T, threshold, tok, n_tok, W, dev_status, (cudaStream_t)stream),
+                     "qsa_dense_select launch");
 }
 
 qsa_status_t qsa_topk_expand(const float* scores, int score_stride, uint32_t* prefix_hist,

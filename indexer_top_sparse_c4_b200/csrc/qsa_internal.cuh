@@ -196,6 +196,8 @@ struct ExpandArgs {
   const int32_t* capture_pos; int T; int32_t* tok; int32_t* n_tok; int W; uint32_t* status;
 };
 cudaError_t launch_expand_select(const ExpandArgs& a, cudaStream_t s);
+cudaError_t launch_dense_select(const int32_t* q_pos, int T, int threshold, int32_t* tok, int32_t* n_tok, int W,
+                                uint32_t* status, cudaStream_t s);
 
 struct AttnArgs {
   const void* q; qsa_dtype_t q_dt; const void* k_pages; const void* v_pages; qsa_dtype_t kv_dt;

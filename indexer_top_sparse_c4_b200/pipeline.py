@@ -19,10 +19,22 @@ from .workloads import GROUP_TOKENS, Workload
 
 
 class QSAStep:
+    """seq_len_threshold (TensorRT-LLM "QSASparseAttentionConfig"): queries
+    whose sequence has at most this many tokens attend densely to all of
+    them; None or a value below the token budget 4*K means the budget, which
+    the Top-K's dense fallback (c <= K) already honours, so no extra launch is
+    made then."""
+
     def __init__(self, w: Workload, prefill: bool | None = None, out_dtype=None,
-                 score_stride: int | None = None, prefix_hist: bool | None = None):
+                 score_stride: int | None = None, prefix_hist: bool | None = None,
+                 seq_len_threshold: int | None = None):
         self.w = w
         dev = w.q.device
+        self.threshold = qsa.qsa_seq_len_threshold(seq_len_threshold, w.K)
+        # an explicit threshold above the budget: dense rows up to that many tokens
+        self.dense_rows = self.threshold > GROUP_TOKENS * w.K
+        if self.dense_rows and self.threshold > w.W:
+            w.W = self.threshold
         self.prefill = (w.T > 64) if prefill is None else prefill
         self.sel_pos = w.capture_pos if w.capture_pos is not None else w.q_pos
         if score_stride is None:
@@ -83,7 +95,8 @@ class QSAStep:
                                        self.n_tok, self.out, workspace=self.ws, **common)
 
     def select(self, stream=None):
-        """Top-K and expansion: one launch when there is no MTP capture."""
+        """Top-K and expansion: one launch when there is no MTP capture; then
+        the dense rows of an explicit sequence-length threshold."""
         w = self.w
         if w.capture_pos is None:
             qsa.qsa_topk_expand(self.scores, w.q_pos, w.K, self.sel, self.n_sel, self.tok, self.n_tok,
@@ -91,12 +104,59 @@ class QSAStep:
         else:
             self.topk(stream)
             self.expand(stream)
+        if self.dense_rows:
+            self.dense_select(self.threshold, stream)
+
+    def dense_select(self, threshold, stream=None):
+        qsa.qsa_dense_select(self.w.q_pos, threshold, self.tok, self.n_tok, dev_status=self.status, stream=stream)
 
     def run(self, stream=None, sm_scale=0.0):
         self.index_scores(stream)
         self.select(stream)
         self.attention(stream, sm_scale)
         return self.out
+
+
+class QSADecodeGraphs:
+    """The two decode graph families of the sequence-length threshold
+    (TensorRT-LLM "QSASparseAttentionConfig",
+    needs_separate_short_long_cuda_graphs): one CUDA graph of a step for
+    batches whose every sequence is at most the threshold -- dense attention
+    over every token, no indexer and no Top-K launched -- and one of the full
+    QSA step (rows at or below the threshold still dense) for the others.
+    The caller updates the step's inputs in place and replays the family
+    its batch needs; the host knows the sequence lengths of its batch."""
+
+    def __init__(self, step: QSAStep, stream=None):
+        if step.prefill or step.w.capture_pos is not None:
+            raise ValueError("decode steps without an MTP capture")
+        self.step = step
+        self.stream = stream if stream is not None else torch.cuda.Stream(step.w.q.device)
+        big = 1 << 30                    # every row dense
+        with torch.cuda.stream(self.stream):
+            step.run()                   # warm-up outside the capture (first-call set-up)
+            step.dense_select(big)
+            step.attention()
+            torch.cuda.synchronize()
+            self.dense = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.dense, stream=self.stream):
+                step.dense_select(big, self.stream)
+                step.attention(self.stream)
+            self.sparse = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.sparse, stream=self.stream):
+                step.run(self.stream)
+
+    def family(self, max_seq_len: int) -> str:
+        return "dense" if max_seq_len <= self.step.threshold else "sparse"
+
+    def replay(self, max_seq_len: int):
+        """Replays the family of a batch whose longest sequence has
+        max_seq_len tokens (on the graphs' stream); returns its name."""
+        fam = self.family(max_seq_len)
+        if fam == "dense" and max_seq_len > self.step.w.W:
+            raise ValueError("a dense batch wider than the step's token lists")
+        (self.dense if fam == "dense" else self.sparse).replay()
+        return fam
 
 
 class QSADraftLoop:

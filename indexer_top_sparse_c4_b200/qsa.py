@@ -29,6 +29,7 @@ ENTRY_POINTS = (
     "qsa_compress_keys",
     "qsa_index_scores_workspace_size", "qsa_index_scores", "qsa_topk_groups_workspace_size",
     "qsa_topk_groups", "qsa_topk_groups_gvr", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
+    "qsa_seq_len_threshold", "qsa_dense_select",
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
     "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
     "qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
@@ -64,6 +65,10 @@ def lib() -> ctypes.CDLL:
     L.qsa_compress_keys_workspace_size.restype = U
     L.qsa_compress_keys.argtypes = [P, I, I, P, P, P, P, I, P, I, I, P, I, I, P, P]
     L.qsa_compress_keys.restype = I
+    L.qsa_seq_len_threshold.argtypes = [I, I]
+    L.qsa_seq_len_threshold.restype = I
+    L.qsa_dense_select.argtypes = [P, I, I, P, P, I, P, P]
+    L.qsa_dense_select.restype = I
     L.qsa_topk_groups_gvr.argtypes = [P, I, P, I, I, P, P, P, P, P]
     L.qsa_topk_groups_gvr.restype = I
     L.qsa_dcp_shard_positions.argtypes = [P, I, I, I, P, P]
@@ -222,6 +227,19 @@ def qsa_topk_groups(scores, q_pos, K, sel, n_sel, workspace=None, dev_status=Non
         _ptr(scores), scores.shape[1], _ptr(prefix_hist), _ptr(q_pos), T, K, _ptr(sel), _ptr(n_sel),
         _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
     return sel, n_sel
+
+
+def qsa_seq_len_threshold(requested, K) -> int:
+    """Tokens at or below which a sequence takes dense attention (None or
+    <= 0: the token budget 4*K; never below it)."""
+    return int(lib().qsa_seq_len_threshold(int(requested or 0), int(K)))
+
+
+def qsa_dense_select(q_pos, threshold, tok, n_tok, dev_status=None, stream=None):
+    T, W = tok.shape
+    _check(lib().qsa_dense_select(_ptr(q_pos), T, int(threshold), _ptr(tok), _ptr(n_tok), W, _ptr(dev_status),
+                                  _stream(stream)))
+    return tok, n_tok
 
 
 def qsa_topk_groups_gvr(scores, q_pos, K, sel, n_sel, path=None, dev_status=None, stream=None):

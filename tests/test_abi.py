@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 8
+    assert L.qsa_abi_version() == 9
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -201,3 +201,14 @@ def test_indexer_write_validation(L):
     assert L.qsa_compress_keys(ok, 128, 4, NULL, NULL, ok, NULL, 128, ok, 0, 4, ok, 1, 4, NULL, NULL) == 1
     assert L.qsa_compress_keys(NULL, 128, 0, NULL, NULL, NULL, NULL, 128, NULL, 0, 4, NULL, 1, 4, NULL, NULL) == 0
     assert L.qsa_compress_keys_workspace_size(2048, 128) == 0
+
+
+def test_seq_len_threshold_resolution(L):
+    """TensorRT-LLM's rule: unset -> the token budget (4 tokens per group of
+    the budget); an explicit value below the budget is raised to it."""
+    assert L.qsa_seq_len_threshold(0, 512) == 2048
+    assert L.qsa_seq_len_threshold(-5, 1024) == 4096
+    assert L.qsa_seq_len_threshold(100, 512) == 2048
+    assert L.qsa_seq_len_threshold(10000, 512) == 10000
+    assert L.qsa_dense_select(NULL, 0, 100, NULL, NULL, 16, NULL, NULL) == 0
+    assert L.qsa_dense_select(NULL, 2, 100, NULL, NULL, 16, NULL, NULL) == 1 and "null" in _err(L)
