@@ -257,10 +257,8 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
         const int kk = j * KS + q4;
         uint32_t af[4];
         if constexpr (FP8) {  // one word = 4 codes = dims 4q4..4q4+3 of the chunk
-          af[0] = e4m3x2_to_f16x2(w0[q4]);
-          af[1] = e4m3x2_to_f16x2(w1[q4]);
-          af[2] = e4m3x2_to_f16x2(w0[q4] >> 16);
-          af[3] = e4m3x2_to_f16x2(w1[q4] >> 16);
+          e4m3x4_to_f16x2x2(w0[q4], af[0], af[2]);
+          e4m3x4_to_f16x2x2(w1[q4], af[1], af[3]);
           mma_f16(sc, af, qb[kk][0], qb[kk][1]);
         } else {              // two words = 4 bf16 = dims 4q4..4q4+3 of the chunk
           af[0] = w0[2 * q4];
@@ -291,9 +289,9 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
       const float mn0 = mx0 > m0 + 8.f ? mx0 : m0;
       const float mn1 = mx1 > m1 + 8.f ? mx1 : m1;
       const float b0 = mn0 == -INFINITY ? 0.f : mn0, b1 = mn1 == -INFINITY ? 0.f : mn1;
-      const float al0 = m0 == -INFINITY ? 0.f : exp2f(m0 - b0);
-      const float al1 = m1 == -INFINITY ? 0.f : exp2f(m1 - b1);
-      const float p0 = exp2f(s0 - b0), p1 = exp2f(s1 - b1), p2 = exp2f(s2 - b0), p3 = exp2f(s3 - b1);
+      const float al0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - b0);
+      const float al1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - b1);
+      const float p0 = fast_exp2(s0 - b0), p1 = fast_exp2(s1 - b1), p2 = fast_exp2(s2 - b0), p3 = fast_exp2(s3 - b1);
       m0 = mn0;
       m1 = mn1;
       l0 = l0 * al0 + p0 + p2;
@@ -331,14 +329,10 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
           const uint32_t hi89 = __byte_perm(vc[wd], vd[wd], 0x7362);
           const int mt = j * MTJ + 2 * wd;
           uint32_t af[4], ag[4];
-          af[0] = e4m3x2_to_f16x2(lo01);
-          af[1] = e4m3x2_to_f16x2(lo01 >> 16);
-          af[2] = e4m3x2_to_f16x2(lo89);
-          af[3] = e4m3x2_to_f16x2(lo89 >> 16);
-          ag[0] = e4m3x2_to_f16x2(hi01);
-          ag[1] = e4m3x2_to_f16x2(hi01 >> 16);
-          ag[2] = e4m3x2_to_f16x2(hi89);
-          ag[3] = e4m3x2_to_f16x2(hi89 >> 16);
+          e4m3x4_to_f16x2x2(lo01, af[0], af[1]);
+          e4m3x4_to_f16x2x2(lo89, af[2], af[3]);
+          e4m3x4_to_f16x2x2(hi01, ag[0], ag[1]);
+          e4m3x4_to_f16x2x2(hi89, ag[2], ag[3]);
           mma_f16(o[mt], af, pb[0], pb[1]);
           mma_f16(o[mt + 1], ag, pb[0], pb[1]);
         } else {

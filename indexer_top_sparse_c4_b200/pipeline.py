@@ -134,9 +134,10 @@ class QSADecodeGraphs:
         self.stream = stream if stream is not None else torch.cuda.Stream(step.w.q.device)
         big = 1 << 30                    # every row dense
         with torch.cuda.stream(self.stream):
-            step.run()                   # warm-up outside the capture (first-call set-up)
-            step.dense_select(big)
-            step.attention()
+            # warm-up outside the capture (first-call set-up of every kernel);
+            # the dense rows of the step's own threshold always fit its lists
+            step.run()
+            step.dense_select(step.threshold)
             torch.cuda.synchronize()
             self.dense = torch.cuda.CUDAGraph()
             with torch.cuda.graph(self.dense, stream=self.stream):
