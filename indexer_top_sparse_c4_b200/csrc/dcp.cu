@@ -133,20 +133,18 @@ __global__ void __launch_bounds__(kMgThreads) dcp_merge_topk_kernel(const float*
     for (int shift = 56; shift >= 0; shift -= 8) {
       for (int b = tid; b < 256; b += kMgThreads) hist[b] = 0;
       __syncthreads();
-      for (int i = tid; i < n; i += kMgThreads) {
-        const uint64_t k = keys[i];
-        if ((k & mask) == prefix) atomicAdd(&hist[(int)((k >> shift) & 0xFF)], 1);
+      for (int base = 0; base < n; base += kMgThreads) {   // one atomic per bin and warp
+        const int i = base + tid;
+        int bin = -1;
+        if (i < n) {
+          const uint64_t k = keys[i];
+          if ((k & mask) == prefix) bin = (int)((k >> shift) & 0xFF);
+        }
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (bin >= 0 && (tid & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
       }
       __syncthreads();
-      if (tid == 0) {   // the bin holding the need-th largest among the matching keys
-        int acc = 0, b = 255;
-        for (; b > 0; --b) {
-          if (acc + hist[b] >= need) break;
-          acc += hist[b];
-        }
-        s_bin = b;
-        s_need = need - acc;
-      }
+      find_bin_from_top(hist, need, &s_bin, &s_need);   // the bin of the need-th largest matching key
       __syncthreads();
       prefix |= (uint64_t)s_bin << shift;
       mask |= 0xFFull << shift;

@@ -125,6 +125,43 @@ constexpr int kPrefixBins = 1 << kPrefixBits;
 constexpr int kPrefixShift = 32 - kPrefixBits;
 static_assert(kPrefixBins == QSA_PREFIX_HIST_BINS, "prefix histogram width");
 
+// ---- radix select helper -------------------------------------------------------
+// The bin (0..255) holding the need-th largest of the counted keys, scanning
+// from the top, and the rank left inside it: warp 0 reads 8 bins per lane,
+// finds the lane by a warp scan from the top, then the bin inside the lane.
+__device__ __forceinline__ void find_bin_from_top(const int* hist, int need, int* s_bin, int* s_need) {
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x >= 32) return;
+  // lane l holds bins 255 - 8l .. 248 - 8l (highest first)
+  int c[8];
+  int sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = hist[255 - 8 * lane - j];
+    sum += c[j];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += y;
+  }
+  const int excl = incl - sum;
+  const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+  const int L = hit ? __ffs(hit) - 1 : 31;
+  if (lane == L) {
+    int acc = excl, b = 255 - 8 * lane;
+    int j = 0;
+    for (; j < 7; ++j) {
+      if (acc + c[j] >= need) break;
+      acc += c[j];
+    }
+    b -= j;
+    *s_bin = b;
+    *s_need = need - acc;
+  }
+}
+
 // ---- programmatic dependent launch (PDL) ----------------------------------------
 // Every kernel of the library is launched with programmatic stream
 // serialisation, so its CTAs may be scheduled while the previous kernel on the

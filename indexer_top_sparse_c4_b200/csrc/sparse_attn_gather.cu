@@ -244,7 +244,9 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
     const bool ok0 = tbl[tb + g] >= 0, ok1 = tbl[tb + g + 8] >= 0;
 
     // ---- S^T = K . Q^T for this warp's head tile (rows g and g+8 share a swizzle)
-    float sc[4] = {0.f, 0.f, 0.f, 0.f};
+    // four independent accumulator chains (k-step kk feeds chain kk % 4): the
+    // MMAs of a chain wait on each other, the chains do not
+    float scc[4][4] = {};
 #pragma unroll
     for (int j = 0; j < KJ; ++j) {
       const int pc = ((4 * j + tq) ^ ga_sw(g)) * 16;
@@ -259,16 +261,20 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
         if constexpr (FP8) {  // one word = 4 codes = dims 4q4..4q4+3 of the chunk
           e4m3x4_to_f16x2x2(w0[q4], af[0], af[2]);
           e4m3x4_to_f16x2x2(w1[q4], af[1], af[3]);
-          mma_f16(sc, af, qb[kk][0], qb[kk][1]);
+          mma_f16(scc[kk & 3], af, qb[kk][0], qb[kk][1]);
         } else {              // two words = 4 bf16 = dims 4q4..4q4+3 of the chunk
           af[0] = w0[2 * q4];
           af[1] = w1[2 * q4];
           af[2] = w0[2 * q4 + 1];
           af[3] = w1[2 * q4 + 1];
-          mma_bf16(sc, af, qb[kk][0], qb[kk][1]);
+          mma_bf16(scc[kk & 3], af, qb[kk][0], qb[kk][1]);
         }
       }
     }
+
+    float sc[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[e] = (scc[0][e] + scc[1][e]) + (scc[2][e] + scc[3][e]);
 
     // ---- online softmax, heads 8u + 2tq (s0, s2) and 8u + 2tq + 1 (s1, s3)
     uint32_t pb[2];

@@ -14,9 +14,11 @@
 //    guess moves (a deeper sample rank when too few, a shallower one when too
 //    many) and the count is taken again, up to three times;
 //  * refine: the >= tau candidates are gathered into shared memory in id
-//    order (a block prefix sum over per-thread counts of contiguous id
-//    ranges) and an exact radix select over at most CAP of them finds the
-//    K-th key; the kept ones are written ascending by a second prefix sum;
+//    order and an exact radix select over at most CAP of them finds the K-th
+//    key; the kept ones are written ascending.  Every pass over ids gives
+//    each warp a contiguous range read 32 consecutive scores at a time
+//    (coalesced); ballots order a warp's hits, and one prefix sum over the
+//    32 warps' counts orders the warps;
 //  * a row whose guesses all fail (e.g. thousands of equal scores) runs the
 //    same radix select over the whole row instead.
 // path[t] (optional) records what happened: 0 dense (c <= K), 1 the first
@@ -82,20 +84,21 @@ __device__ uint32_t gv_select(Get get, int m, int r, GvShared& sh, int* above) {
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int b = threadIdx.x; b < 256; b += kGvThreads) sh.hist[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < m; i += kGvThreads) {
-      const uint32_t k = get(i);
-      if ((k & mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 0xFF], 1);
+    // keys of a warp that fall in the same bin are counted with one atomic
+    // (the top digits of a row's scores are mostly equal: per-key atomics on
+    // one bin would serialise)
+    for (int base = 0; base < m; base += kGvThreads) {
+      const int i = base + threadIdx.x;
+      int bin = -1;
+      if (i < m) {
+        const uint32_t k = get(i);
+        if ((k & mask) == prefix) bin = (int)((k >> shift) & 0xFF);
+      }
+      const unsigned peers = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && (int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], __popc(peers));
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int acc = 0, b = 255;
-      for (; b > 0; --b) {
-        if (acc + sh.hist[b] >= need) break;
-        acc += sh.hist[b];
-      }
-      sh.s_bin = b;
-      sh.s_need = need - acc;
-    }
+    find_bin_from_top(sh.hist, need, &sh.s_bin, &sh.s_need);
     __syncthreads();
     prefix |= (uint32_t)sh.s_bin << shift;
     mask |= 0xFFu << shift;
@@ -104,6 +107,86 @@ __device__ uint32_t gv_select(Get get, int m, int r, GvShared& sh, int* above) {
   }
   *above = r - need;   // keys strictly greater than the r-th largest
   return prefix;
+}
+
+// A warp's contiguous share [lo, hi) of n ids (multiples of 32 wide).
+__device__ __forceinline__ void gv_warp_range(int n, int& lo, int& hi) {
+  const int warp = threadIdx.x >> 5;
+  const int per = ((n + kGvThreads / 32 - 1) / (kGvThreads / 32) + 31) / 32 * 32;
+  lo = warp * per < n ? warp * per : n;
+  hi = lo + per < n ? lo + per : n;
+}
+
+constexpr int kGvUnroll = 8;   // 32-wide steps a warp loads before it tests them
+
+// Ids i in [0, n) whose key get(i) satisfies pred(key), in id order:
+// emit(position, i, key).  Returns the total.  Every thread of the block
+// calls it.  Each warp loads kGvUnroll steps of 32 consecutive keys before it
+// tests them, so a warp has that many loads in flight.
+template <typename Get, typename Pred, typename Emit>
+__device__ int gv_ordered(int n, Get get, Pred pred, Emit emit, GvShared& sh) {
+  const int lane = threadIdx.x & 31;
+  int lo, hi;
+  gv_warp_range(n, lo, hi);
+  int cnt = 0;
+  for (int k = lo; k < hi; k += 32 * kGvUnroll) {
+    uint32_t v[kGvUnroll];
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      v[u] = i < hi ? get(i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, i < hi && pred(v[u])));
+    }
+  }
+  int total;
+  // one value per warp enters the block scan (lane 0 carries it)
+  int base = gv_scan(lane == 0 ? cnt : 0, sh, &total);
+  base = __shfl_sync(0xffffffffu, base, 0);
+  const unsigned below = (1u << lane) - 1u;
+  for (int k = lo; k < hi; k += 32 * kGvUnroll) {
+    uint32_t v[kGvUnroll];
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      v[u] = i < hi ? get(i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      const bool f = i < hi && pred(v[u]);
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+      if (f) emit(base + __popc(m & below), i, v[u]);
+      base += __popc(m);
+    }
+  }
+  return total;
+}
+
+// How many ids i in [0, n) have pred(get(i)) (coalesced warp ranges).
+template <typename Get, typename Pred>
+__device__ int gv_count(int n, Get get, Pred pred, GvShared& sh) {
+  const int lane = threadIdx.x & 31;
+  int lo, hi;
+  gv_warp_range(n, lo, hi);
+  int cnt = 0;
+  for (int k = lo; k < hi; k += 32 * kGvUnroll) {
+    uint32_t v[kGvUnroll];
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      v[u] = i < hi ? get(i) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kGvUnroll; ++u) {
+      const int i = k + 32 * u + lane;
+      cnt += __popc(__ballot_sync(0xffffffffu, i < hi && pred(v[u])));
+    }
+  }
+  return gv_sum(lane == 0 ? cnt : 0, sh);
 }
 
 __global__ void __launch_bounds__(kGvThreads, 1)
@@ -136,19 +219,13 @@ __global__ void __launch_bounds__(kGvThreads, 1)
   __syncthreads();
   int r = (int)(((long long)(K + K / 4 + 32) * S + c - 1) / c);
   r = r < 1 ? 1 : (r > S ? S : r);
-  // each thread owns a contiguous range of ids: prefix sums give id order
-  const int per = (c + kGvThreads - 1) / kGvThreads;
-  const int lo = tid * per < c ? tid * per : c;
-  const int hi = lo + per < c ? lo + per : c;
 
   int count = -1, tries = 0, dummy;
   uint32_t tau = 0u;
   while (tries < kGvTries) {
     tau = gv_select([&](int i) { return sh.sample[i]; }, S, r, sh, &dummy);
     // ---- verify: how many of the row's keys reach the guess
-    int mine = 0;
-    for (int i = lo; i < hi; ++i) mine += key_at(i) >= tau;
-    count = gv_sum(mine, sh);
+    count = gv_count(c, key_at, [&](uint32_t k) { return k >= tau; }, sh);
     ++tries;
     if (count >= K && count <= kGvCap) break;
     if (count < K) {
@@ -161,83 +238,52 @@ __global__ void __launch_bounds__(kGvThreads, 1)
     count = -1;
   }
 
-  if (count >= K && count <= kGvCap) {
+  int tk_above;
+  uint32_t tk;
+  bool from_buffer = count >= K && count <= kGvCap;
+  if (from_buffer) {
     // ---- refine: gather the candidates in id order, then an exact select among them
-    int mine = 0;
-    for (int i = lo; i < hi; ++i) mine += key_at(i) >= tau;
-    int total;
-    int pos = gv_scan(mine, sh, &total);
-    for (int i = lo; i < hi; ++i) {
-      const uint32_t k = key_at(i);
-      if (k >= tau) {
-        sh.ckey[pos] = k;
-        sh.cid[pos] = i;
-        ++pos;
-      }
-    }
+    const int total = gv_ordered(c, key_at, [&](uint32_t k) { return k >= tau; },
+                                 [&](int pos, int i, uint32_t k) {
+                                   sh.ckey[pos] = k;
+                                   sh.cid[pos] = i;
+                                 },
+                                 sh);
     __syncthreads();
-    int above;
-    const uint32_t tk = gv_select([&](int i) { return sh.ckey[i]; }, total, K, sh, &above);
-    const int need = K - above;   // keys equal to tk that are kept: the lowest ids among them
-    // kept = key > tk, or key == tk among the first `need` equal keys in id order
-    const int per2 = (total + kGvThreads - 1) / kGvThreads;
-    const int a0 = tid * per2 < total ? tid * per2 : total;
-    const int a1 = a0 + per2 < total ? a0 + per2 : total;
-    int eq = 0;
-    for (int i = a0; i < a1; ++i) eq += sh.ckey[i] == tk;
-    int eq_total;
-    int eq_before = gv_scan(eq, sh, &eq_total);
-    int kept = 0;
-    {
-      int e = eq_before;
-      for (int i = a0; i < a1; ++i) {
-        const uint32_t k = sh.ckey[i];
-        if (k > tk || (k == tk && e++ < need)) ++kept;
-      }
-    }
-    int kt;
-    int opos = gv_scan(kept, sh, &kt);
-    {
-      int e = eq_before;
-      for (int i = a0; i < a1; ++i) {
-        const uint32_t k = sh.ckey[i];
-        if (k > tk || (k == tk && e++ < need)) out[opos++] = sh.cid[i];
-      }
-    }
-    if (tid == 0) {
-      n_sel[t] = K;
-      if (path) path[t] = tries == 1 ? 1 : 2;
-    }
+    count = total;
+    tk = gv_select([&](int i) { return sh.ckey[i]; }, total, K, sh, &tk_above);
   } else {
     // ---- fallback: the exact radix select over the whole row
-    int above;
-    const uint32_t tk = gv_select(key_at, c, K, sh, &above);
-    const int need = K - above;
-    int eq = 0;
-    for (int i = lo; i < hi; ++i) eq += key_at(i) == tk;
-    int eq_total;
-    const int eq_before = gv_scan(eq, sh, &eq_total);
-    int kept = 0;
-    {
-      int e = eq_before;
-      for (int i = lo; i < hi; ++i) {
-        const uint32_t k = key_at(i);
-        if (k > tk || (k == tk && e++ < need)) ++kept;
-      }
-    }
-    int kt;
-    int opos = gv_scan(kept, sh, &kt);
-    {
-      int e = eq_before;
-      for (int i = lo; i < hi; ++i) {
-        const uint32_t k = key_at(i);
-        if (k > tk || (k == tk && e++ < need)) out[opos++] = i;
-      }
-    }
-    if (tid == 0) {
-      n_sel[t] = K;
-      if (path) path[t] = 3;
-    }
+    tk = gv_select(key_at, c, K, sh, &tk_above);
+  }
+  // keys equal to tk: the `need` lowest ids among them are kept
+  const int need = K - tk_above;
+  const int n = from_buffer ? count : c;
+  auto key_of = [&](int i) { return from_buffer ? sh.ckey[i] : key_at(i); };
+  auto id_of = [&](int i) { return from_buffer ? sh.cid[i] : i; };
+  // the rank of each equal key among the equal keys, in id order: the first
+  // `need` of them are kept; a first ordered pass records the cut-off id
+  if (tid == 0) sh.s_count = 0x7fffffff;
+  __syncthreads();
+  gv_ordered(n, key_of, [&](uint32_t k) { return k == tk; },
+             [&](int pos, int i, uint32_t) {
+               if (pos == need - 1) sh.s_count = i;   // the last equal key kept
+             },
+             sh);
+  __syncthreads();
+  const int last_eq = sh.s_count;
+  // kept: above tk, or equal to it and not past the last equal key kept
+  // (equal keys past it are read as 0, below every real key)
+  gv_ordered(n, [&](int i) {
+               const uint32_t k = key_of(i);
+               // keys equal to tk past the cut-off are sent below tk
+               return (k == tk && i > last_eq) ? 0u : k;
+             },
+             [&](uint32_t k) { return k >= tk && k != 0u; },
+             [&](int pos, int i, uint32_t) { out[pos] = id_of(i); }, sh);
+  if (tid == 0) {
+    n_sel[t] = K;
+    if (path) path[t] = from_buffer ? (tries == 1 ? 1 : 2) : 3;
   }
 }
 
