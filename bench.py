@@ -452,9 +452,115 @@ def gpu_arm(args):
         line["mtp"] = mtp_summary(device, stream, args.seed, 20)
     if args.prefill and ws == 1:
         line["prefill"] = prefill_summary(device, stream, args.seed, 3)
+    if args.features and ws == 1:
+        line["features"] = features_summary(device, stream, args.seed)
     if host_copy is not None:
         line["cpu_baseline"] = cpu_baseline(host_copy, w0, args.cpu_seconds)
     return line
+
+
+def graph_us(fn, reps, stream):
+    """Device time per call of fn(i), i < reps, from one CUDA graph of the
+    reps calls (CUDA events on the graph's stream)."""
+    with torch.cuda.stream(stream):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                fn(i)
+        g.replay()
+        ms = replay_ms(g)
+        del g
+    return ms / reps * 1e3
+
+
+def features_summary(device, stream, seed):
+    """The entry points beyond the four-stage decode step, each timed on the
+    device (graphs of launches): the guess-verify-refine Top-K, the indexer
+    projection and C4 compressed-key write, the dense and sparse graph
+    families of the sequence-length threshold, and sequence-sharded decode
+    emulated on this one GPU."""
+    from indexer_top_sparse_c4_b200 import qsa, workloads as wl
+    from indexer_top_sparse_c4_b200.dcp import QSADcpDecode
+    from indexer_top_sparse_c4_b200.pipeline import QSADecodeGraphs, QSAStep
+    out = {}
+    reps = 20
+    # ---- Top-K on the B8 x 262,144 rows: GVR (no hint), radix without and with the scan's histogram
+    topk = {}
+    for K in (512, 2048):
+        sets = [QSAStep(wl.b8_262k(K=K, device=device, seed=seed + i)) for i in (0, 1)]
+        for st in sets:
+            st.run()
+        torch.cuda.synchronize()
+        path = torch.empty((8,), dtype=torch.int32, device=device)
+        g = graph_us(lambda i: qsa.qsa_topk_groups_gvr(sets[i % 2].scores, sets[i % 2].w.q_pos, K, sets[i % 2].sel,
+                                                      sets[i % 2].n_sel, path=path), reps, stream)
+        r = graph_us(lambda i: qsa.qsa_topk_groups(sets[i % 2].scores, sets[i % 2].w.q_pos, K, sets[i % 2].sel,
+                                                   sets[i % 2].n_sel), reps, stream)
+        scan = graph_us(lambda i: sets[i % 2].index_scores(), reps, stream)
+        both = graph_us(lambda i: (sets[i % 2].index_scores(), sets[i % 2].topk()), reps, stream)
+        for st in sets:
+            st.prefix_hist.zero_()
+        topk[str(K)] = {"gvr_us": round(g, 2), "radix_no_hint_us": round(r, 2),
+                        "radix_with_scan_histogram_us": round(both - scan, 2),
+                        "gvr_paths": sorted(set(path.tolist()))}
+        del sets
+    out["topk_b8_262k"] = topk
+    # ---- indexer projection and compressed-key write (hidden 5,120, 4 x 128 indexer)
+    H, N, D_I = 5120, 4 * 128 + 4 + 128, 128
+    w, wphi, bias = wl.indexer_weights(H, 4, D_I, seed=seed, device=device)
+    proj = {}
+    for T in (8, 8192):
+        x = wl.hidden_states(T, H, seed=seed + 1, device=device)
+        y = torch.empty((T, N), dtype=torch.float32, device=device)
+        us = graph_us(lambda i: qsa.qsa_indexer_project(x, w, y), reps, stream)
+        flop = 2.0 * T * H * N
+        proj[str(T)] = {"us": round(us, 2), "tflops": round(flop / us / 1e6, 1),
+                        "weight_gbs": round(N * H * 2 / us / 1e3, 1)}
+    pages = torch.zeros((8192 // 64 + 1, 16, D_I), dtype=torch.float32, device=device)
+    pt = torch.arange(pages.shape[0], dtype=torch.int32, device=device).view(1, -1)
+    g_id = torch.arange(8192 // 4, dtype=torch.int32, device=device)
+    cmp_us = graph_us(lambda i: qsa.qsa_compress_keys(y[:, 4 * 128 + 4:], g_id, wphi, pages, pt, bias=bias), reps,
+                      stream)
+    out["indexer_write"] = {"projection": proj, "bound": {"8": "hbm (the weights)", "8192": "tensor"},
+                            "compress_2048_groups_us": round(cmp_us, 2)}
+    # ---- graph families of the sequence-length threshold (B8, 16,384 context, threshold 6,000)
+    pos = torch.full((8,), 16383, dtype=torch.int32)
+    wt = wl.make("thr", B=8, ctx=16384, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype="fp8",
+                 q_dtype="bf16", dist="peaked", seed=seed, device=device, q_pos=pos, q_req=torch.arange(8))
+    st = QSAStep(wt, seq_len_threshold=6000)
+    fams = QSADecodeGraphs(st, stream)
+
+    def replays_us(name, max_len):
+        with torch.cuda.stream(fams.stream):
+            fams.replay(max_len)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                assert fams.replay(max_len) == name
+            b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e3
+
+    sparse_us = replays_us("sparse", 16384)
+    wt.q_pos.fill_(5999)
+    dense_us = replays_us("dense", 6000)
+    out["seq_len_threshold"] = {"threshold": st.threshold, "sparse_family_step_us": round(sparse_us, 2),
+                                "dense_family_step_us_at_6000_tokens": round(dense_us, 2)}
+    del fams, st, wt
+    # ---- sequence-sharded decode emulated on one GPU (all shards in turn, merges included)
+    dcp = {}
+    wd = wl.b8_262k(K=512, device=device, seed=seed)
+    for R in (2, 4):
+        d = QSADcpDecode(wd, R)
+        us = graph_us(lambda i: d.run(), 5, stream)
+        dcp[str(R)] = {"emulated_step_us": round(us, 2),
+                       "records_bytes_per_rank": 8 * wd.K * 8, "partials_bytes_per_rank": 8 * 16 * 256 * 4 + 8 * 16 * 4}
+        del d
+    out["dcp_b8_262k_k512"] = {"shards": dcp, "note": "one GPU runs every shard in turn; no collective crosses "
+                                                      "NVLink in this measurement"}
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---- the prefill chunk ------------------------------------------------------------------
@@ -696,6 +802,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-mtp", dest="mtp", action="store_false",
                     help="skip the MTP draft loop (index sharing) line")
+    ap.add_argument("--no-features", dest="features", action="store_false",
+                    help="leave out the timings of the entry points beyond the decode step")
     ap.add_argument("--no-prefill", dest="prefill", action="store_false",
                     help="leave out the prefill-chunk summary of the decode line")
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
