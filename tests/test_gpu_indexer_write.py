@@ -28,10 +28,11 @@ def _projection_bound(x, w):
     return SCORE_REL * (np.abs(values_f64(x)) @ np.abs(values_f64(w)).T)
 
 
-def _check_projection(q, oracle, T, H, x_dt="bf16", w_dt="bf16", rows=None, seed=0):
+def _check_projection(q, oracle, T, H, x_dt="bf16", w_dt="bf16", rows=None, seed=0, n_rows=N):
     x = wl.hidden_states(T, H, seed=seed, device="cuda", dtype=x_dt)
     w, _, _ = wl.indexer_weights(H, H_I, D_I, seed=seed + 1, device="cuda", dtype=w_dt)
-    y = torch.full((T, N), float("nan"), dtype=torch.float32, device="cuda")
+    w = w[:n_rows]
+    y = torch.full((T, n_rows), float("nan"), dtype=torch.float32, device="cuda")
     status = torch.zeros((1,), dtype=torch.int32, device="cuda")
     q.qsa_indexer_project(x, w, y, dev_status=status)
     torch.cuda.synchronize()
@@ -54,6 +55,16 @@ def test_projection_decode_gemv(q, oracle, T):
     _check_projection(q, oracle, T, 512, x_dt="f32", w_dt="f32", seed=5)
 
 
+@pytest.mark.parametrize("T", [3, 11])
+def test_projection_gemv_hidden_chunks_and_ragged_rows(q, oracle, T):
+    """Hidden sizes past one chunk of the GEMV's register-staged row (6,144
+    columns for BF16 w, 4,096 for FP32 w), each with a ragged last chunk, and
+    a row count that leaves the last CTA's four rows partly empty."""
+    _check_projection(q, oracle, T, 8200, seed=11)
+    _check_projection(q, oracle, T, 4104, x_dt="f32", w_dt="f32", seed=13)
+    _check_projection(q, oracle, T, 2048, seed=15, n_rows=641)
+
+
 def test_projection_prefill_tensor_cores_ragged(q, oracle):
     """The tcgen05 GEMM on a token count and a row count that are not
     multiples of its 128 x 128 tiles: every row checked."""
@@ -67,21 +78,22 @@ def test_projection_prefill_chunk_sampled(q, oracle):
     _check_projection(q, oracle, 8192, 5120, rows=rows)
 
 
-def _pages_with_sentinel(num_pages, dt):
+def _pages_with_sentinel(num_pages, dt, d=D_I):
     if dt == "f32":
-        return torch.full((num_pages, 16, D_I), 7.0, dtype=torch.float32, device="cuda")
-    return torch.full((num_pages, 16, D_I), 7.0, dtype=torch.bfloat16, device="cuda")
+        return torch.full((num_pages, 16, d), 7.0, dtype=torch.float32, device="cuda")
+    return torch.full((num_pages, 16, d), 7.0, dtype=torch.bfloat16, device="cuda")
 
 
-def _check_compress(q, oracle, k_tok, g_id, g_req, pt, num_pages, dt, seed=0):
-    _, wphi, bias = wl.indexer_weights(256, H_I, D_I, seed=seed, device="cuda")
-    pages = _pages_with_sentinel(num_pages, dt)
+def _check_compress(q, oracle, k_tok, g_id, g_req, pt, num_pages, dt, seed=0, weights=None):
+    d = k_tok.shape[1]
+    _, wphi, bias = wl.indexer_weights(256, H_I, d, seed=seed, device="cuda") if weights is None else weights
+    pages = _pages_with_sentinel(num_pages, dt, d)
     status = torch.zeros((1,), dtype=torch.int32, device="cuda")
     q.qsa_compress_keys(k_tok, g_id, wphi, pages, pt, g_req=g_req, bias=bias, dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    want = host(_pages_with_sentinel(num_pages, dt))
-    kt = host(k_tok.contiguous()).reshape(-1, 4, D_I)
+    want = host(_pages_with_sentinel(num_pages, dt, d))
+    kt = host(k_tok.contiguous()).reshape(-1, 4, d)
     skipped = oracle.compress_keys(kt, host(g_id), host(wphi), want, host(pt),
                                    g_req=None if g_req is None else host(g_req), bias=host(bias))
     assert skipped == 0
@@ -123,6 +135,27 @@ def test_compress_prefill_chunk_in_place(q, oracle, dt):
     # the chunk follows a 1,024-token prefix: its groups are 256 .. 767 (logical pages 16 .. 47)
     g_id = torch.arange(256, 256 + T // 4, dtype=torch.int32, device="cuda")
     _check_compress(q, oracle, k_tok, g_id, None, pt, pages_per_req, dt)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128])
+def test_compress_dims_unaligned_operands_ragged_groups(q, oracle, d):
+    """Every built D_I, 37 groups (two full CTAs of 16 and a ragged third),
+    token-key rows at an odd stride and a W_phi that does not start on a
+    16-byte boundary: the 4-byte copy paths."""
+    n = 37
+    gen = torch.Generator(device="cpu").manual_seed(40 + d)
+    buf = torch.randn((4 * n, d + 3), generator=gen).cuda()
+    k_tok = buf[:, :d]                                     # row stride d + 3
+    _, wphi, bias = wl.indexer_weights(256, H_I, d, seed=41, device="cuda")
+    raw = torch.empty((wphi.numel() + 1,), dtype=torch.float32, device="cuda")
+    wphi_odd = raw[1:].view(wphi.shape)
+    wphi_odd.copy_(wphi)
+    assert wphi_odd.data_ptr() % 16 != 0 and k_tok.stride(0) % 4 != 0
+    P = 8
+    pt = torch.randperm(P, generator=gen).to(torch.int32).view(1, -1).cuda()
+    g_id = torch.randperm(P * 16, generator=gen)[:n].to(torch.int32).cuda()
+    _check_compress(q, oracle, k_tok, g_id, None, pt, P, "f32", weights=(None, wphi_odd, bias))
+    _check_compress(q, oracle, k_tok, g_id, None, pt, P, "bf16", weights=(None, wphi_odd, bias))
 
 
 def test_compress_decode_ring(q, oracle):
