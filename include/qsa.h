@@ -395,6 +395,24 @@ QSA_API qsa_status_t qsa_dcp_merge_attn(const float* o_parts, const float* lse_p
 QSA_API qsa_status_t qsa_get_device_status(uint32_t* dev_status, uint32_t* bits_out, int clear,
                                            qsa_stream_t stream);
 
+/* Self-test of the bounded wait that every TMA / tensor-core kernel of this
+ * library uses for its mbarrier phases (the error channel above, for a wait
+ * that never completes).  One CTA of two warps: warp 0 puts a 16-byte bulk
+ * copy in flight on one barrier, then waits on a second barrier that nothing
+ * arrives at, with a limit of limit_us microseconds (1 .. 1,000,000); when it
+ * runs out the warp sets the CTA's abort flag and ORs QSA_DEV_TIMEOUT into
+ * *dev_status.  Warp 1 waits on the same barrier with a limit one second
+ * longer and must be released by the abort flag instead.  Warp 0 then drains
+ * the bulk copy (bounded too) before the CTA exits.  No fault, trap or hang:
+ * the context stays usable.  report (device memory, 6 x uint32, written):
+ *   [0] warp 0's wait result (0: timed out), [1] warp 1's wait result
+ *   (0: released), [2] warp 0's wait in microseconds, [3] warp 1's,
+ *   [4] 1 when the drain saw the copy land, [5] 1 when its 16 bytes match.
+ * dev_status must not be NULL.  QSA_ERR_INVALID_ARG for a NULL pointer or a
+ * limit out of range. */
+QSA_API qsa_status_t qsa_selftest_bounded_wait(uint32_t limit_us, uint32_t* dev_status, uint32_t* report,
+                                               qsa_stream_t stream);
+
 /* Human-readable message for the last non-OK status returned on this thread. */
 QSA_API const char* qsa_last_error_string(void);
 /* Static name of a status code. */
@@ -405,7 +423,8 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * status codes QSA_ERR_DEVICE_INDEX / QSA_ERR_TIMEOUT, qsa_get_device_status
  * and a workspace query for every stage; 6: qsa_indexer_project and
  * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*; 8:
- * qsa_topk_groups_gvr; 9: qsa_seq_len_threshold and qsa_dense_select). */
+ * qsa_topk_groups_gvr; 9: qsa_seq_len_threshold and qsa_dense_select; 10:
+ * qsa_selftest_bounded_wait). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -43,12 +43,12 @@ __device__ __forceinline__ unsigned long long gtimer() {
 // Bounded wait for the phase with the given parity; false (and the abort flag
 // set, QSA_DEV_TIMEOUT raised) when it does not come.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status) {
+                                          uint32_t* status, unsigned long long limit_ns = kWaitLimitNs) {
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(b, parity)) return true;
     if (*abort_flag) return false;
-    if ((i & 15u) == 15u && gtimer() - t0 > kWaitLimitNs) break;
+    if ((i & 15u) == 15u && gtimer() - t0 > limit_ns) break;
   }
   *abort_flag = 1;
   flag(status, QSA_DEV_TIMEOUT);
@@ -57,11 +57,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
 // After an abort: wait, with its own bound and whatever the abort flag says,
 // for a phase this thread armed, so that no copy or MMA still writes shared
 // memory or TMEM when the CTA leaves.
-__device__ __forceinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+__device__ __forceinline__ bool mbar_drain(uint64_t* b, uint32_t parity) {
   const unsigned long long t0 = gtimer();
   for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(b, parity)) return;
-    if ((i & 15u) == 15u && gtimer() - t0 > kWaitLimitNs) return;
+    if (mbar_try_wait(b, parity)) return true;
+    if ((i & 15u) == 15u && gtimer() - t0 > kWaitLimitNs) return false;
   }
 }
 

@@ -97,7 +97,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 9; }
+int qsa_abi_version(void) { return 10; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -137,6 +137,14 @@ qsa_status_t qsa_get_device_status(uint32_t* dev_status, uint32_t* bits_out, int
                 (bits & QSA_DEV_BAD_GROUP) ? "group " : "", (bits & QSA_DEV_ROW_RANGE) ? "row-range " : "",
                 (bits & QSA_DEV_BAD_REQUEST) ? "request" : "");
   return QSA_OK;
+}
+
+qsa_status_t qsa_selftest_bounded_wait(uint32_t limit_us, uint32_t* dev_status, uint32_t* report,
+                                       qsa_stream_t stream) {
+  REQUIRE(dev_status && report, "null pointer argument");
+  REQUIRE(limit_us >= 1 && limit_us <= 1000000, "limit_us must be in 1 .. 1,000,000 (got %u)", limit_us);
+  return cuda_status(qsa::launch_selftest_wait(limit_us, dev_status, report, (cudaStream_t)stream),
+                     "qsa_selftest_bounded_wait launch");
 }
 
 size_t qsa_indexer_project_workspace_size(int T, int H, int N) {
@@ -411,7 +419,7 @@ qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void
   qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
                   pt_rows, pt_stride, q_req, tok, n_tok, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
                   dev_status};
-  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{1, 1, true, false}, nullptr, (cudaStream_t)stream,
+  return cuda_status(qsa::launch_sparse_attn(a, qsa::DecodePlan{}, nullptr, (cudaStream_t)stream,
                                              false),
                      "qsa_sparse_attn_prefill launch");
 }

@@ -242,20 +242,17 @@ struct AttnArgs {
   const int32_t* q_req; const int32_t* tok; const int32_t* n_tok; int W, T, Hq, Hkv, D;
   float sm_scale; void* out; qsa_dtype_t out_dt; float* lse; uint32_t* status;
 };
-// How a decode call is spread over the GPU: clusters of `cl` CTAs per
-// (query, KV head) merged on chip, and `s` cluster groups whose partial
-// (o, max, sum) go through the workspace to the combine kernel when s > 1.
 // Plan of the decode kernel that spreads each (query, KV head) row over S
 // CTAs of C token slots each; with S > 1 the combine kernel merges the S
 // partials of a row.
 struct GatherPlan {
   int S, C;
 };
+// How a decode call is spread over the GPU.
 struct DecodePlan {
-  int cl, s;
-  bool stream;   // tensor-core path: one CTA streams a whole row (no split)
-  bool cluster;  // tensor-core path: one cluster of cl CTAs per row, merged on chip
-  bool gather = false;  // tensor-core path: the gather kernel with plan gp; s = gp.S partials per row
+  int s = 1;             // partials per row merged by the combine kernel (1: none)
+  bool stream = false;   // tensor-core path: one warp streams each (query, KV head) row
+  bool gather = false;   // tensor-core path: the gather kernel with plan gp (s = gp.S)
   GatherPlan gp{1, 16};
 };
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
@@ -265,22 +262,12 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits);
 cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
                                bool decode);
 
-// Tensor-core decode kernel (BF16 / FP8 caches, D in {128, 256}, <= 8 query
-// heads per KV head); same partial / output contract as the general kernel.
+// Tensor-core attention kernels (BF16 / FP8 caches, D in {128, 256}, <= 16
+// query heads per KV head).
 bool attn_mma_supported(const AttnArgs& a);
-// Decode kernel with one thread-block cluster of cl CTAs per (query, KV head)
-// row: no workspace, no combine.  Token slots one pass of the kernel covers
-// per warp step (larger rows take several steps).
-int attn_cluster_tokens_per_round(qsa_dtype_t kv_dt, int D, int cl);
 // Many rows: one warp per (query, KV head) row with all its query heads,
 // K/V streamed through a per-warp cp.async ring.
 cudaError_t launch_sparse_attn_prefill_rows(const AttnArgs& a, float qk_scale_log2, float vmul, cudaStream_t s);
-cudaError_t launch_sparse_attn_cluster(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
-                                       cudaStream_t s);
-// Decode kernel for rows too long for one cluster: one 16-token tile per
-// warp, attn_tile_tokens() token slots per CTA, clusters of cl CTAs merged on
-// chip, cluster groups merged by the combine kernel.
-int attn_tile_tokens();
 // Decode kernel for few rows on every SM: rows split into chunks of one CTA
 // each (one wave, one CTA per SM), token rows resolved once per chunk, K/V
 // streamed through per-slot cp.async rings (sparse_attn_gather.cu).
@@ -288,8 +275,6 @@ bool attn_gather_supported(const AttnArgs& a);
 GatherPlan attn_gather_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt);
 cudaError_t launch_sparse_attn_gather(const AttnArgs& a, float qk_scale_log2, float vmul, const GatherPlan& p,
                                       void* ws, cudaStream_t s);
-cudaError_t launch_sparse_attn_tile(const AttnArgs& a, float qk_scale_log2, float vmul, int cl,
-                                    int s, void* ws, cudaStream_t stream);
 
 // Indexer projection y[T, N] = x[T, H] . w[N, H]^T (indexer_write.cu): a GEMV
 // for few tokens, a tcgen05 GEMM for BF16 prefill chunks.
@@ -305,6 +290,9 @@ struct CompressArgs {
   const int32_t* page_table; int pt_rows, pt_stride; uint32_t* status;
 };
 cudaError_t launch_compress_keys(const CompressArgs& c, qsa_dtype_t k_dt, cudaStream_t s);
+
+// Self-test of the bounded mbarrier wait (selftest.cu).
+cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, uint32_t* report, cudaStream_t s);
 
 // Guess-verify-refine Top-K with self-sampling (topk_gvr.cu).
 bool topk_gvr_budget(int K);

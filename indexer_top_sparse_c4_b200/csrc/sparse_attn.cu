@@ -290,38 +290,27 @@ cudaError_t launch_q(const AttnArgs& a, const AttnScales& sc, int splits, void* 
 
 }  // namespace
 
+bool attn_mma_supported(const AttnArgs& a) {
+  return (a.kv_dt == QSA_BF16 || a.kv_dt == QSA_FP8_E4M3) && (a.D == 128 || a.D == 256) &&
+         a.Hq / a.Hkv <= 16;
+}
+
 DecodePlan attn_decode_plan(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt) {
   AttnArgs probe{};
   probe.kv_dt = kv_dt;
   probe.D = D;
   probe.Hq = Hq;
   probe.Hkv = Hkv > 0 ? Hkv : 1;
-  DecodePlan p{1, 1, false, false};
+  DecodePlan p;
   if (attn_gather_supported(probe) && T * probe.Hkv < 148) {
-    // few (query, KV head) rows: every row spread over CTAs on all SMs, their
-    // partials merged by the combine kernel
+    // fewer (query, KV head) rows than SMs: every row spread over CTAs on all
+    // SMs, their partials merged by the combine kernel
     p.gather = true;
     p.gp = attn_gather_plan(T, Hq, probe.Hkv, D, W, kv_dt);
     p.s = p.gp.S;
   } else if (attn_mma_supported(probe)) {
-    const int halves = probe.Hq / probe.Hkv > 8 ? 2 : 1;  // CTAs per KV head
-    const int ctas_per_chunk = T * probe.Hkv * halves;
-    int cl = 8;  // the largest cluster that keeps every row's cluster resident at once
-    while (cl > 1 && ctas_per_chunk * cl > 148) cl >>= 1;
-    const int rounds = (W + attn_cluster_tokens_per_round(kv_dt, D, cl) - 1) /
-                       attn_cluster_tokens_per_round(kv_dt, D, cl);
-    if (ctas_per_chunk >= 148) {
-      // enough (query, KV head) rows to fill the GPU: one CTA streams each row
-      p.stream = true;
-    } else if (rounds <= 3) {
-      // a cluster covers a whole row in at most three steps per warp
-      p.cluster = true;
-      p.cl = cl;
-    } else {
-      // small decode batch: one CTA per 64 token slots, partials through the
-      // workspace to the combine kernel
-      p.s = (W + attn_tile_tokens() - 1) / attn_tile_tokens();
-    }
+    // enough rows to fill the GPU: one warp streams each row
+    p.stream = true;
   } else {
     // general kernel: enough splits to spread small batches over the GPU
     const int rows = T * Hkv > 0 ? T * Hkv : 1;
@@ -340,7 +329,10 @@ size_t attn_decode_ws_bytes(int T, int Hq, int D, int splits) {
 
 cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cudaStream_t s,
                                bool decode) {
-  if (!decode) plan = DecodePlan{1, 1, true, false};
+  if (!decode) {
+    plan = DecodePlan{};
+    plan.stream = true;
+  }
   const int splits = plan.s;
   if (a.T == 0) return cudaSuccess;
   const double scale = a.sm_scale > 0.f ? (double)a.sm_scale : 1.0 / sqrt((double)a.D);
@@ -351,10 +343,8 @@ cudaError_t launch_sparse_attn(const AttnArgs& a, DecodePlan plan, void* ws, cud
   cudaError_t e;
   if (plan.gather) {
     e = launch_sparse_attn_gather(a, sc.qk, sc.vmul, plan.gp, ws, s);
-  } else if (attn_mma_supported(a)) {
-    e = plan.stream    ? launch_sparse_attn_prefill_rows(a, sc.qk, sc.vmul, s)
-        : plan.cluster ? launch_sparse_attn_cluster(a, sc.qk, sc.vmul, plan.cl, s)
-                       : launch_sparse_attn_tile(a, sc.qk, sc.vmul, plan.cl, splits, ws, s);
+  } else if (plan.stream && attn_mma_supported(a)) {
+    e = launch_sparse_attn_prefill_rows(a, sc.qk, sc.vmul, s);
   } else {
     switch (a.D) {
       case 64: e = launch_q<64>(a, sc, splits, ws, s); break;

@@ -33,7 +33,7 @@ ENTRY_POINTS = (
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
     "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
     "qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
-    "qsa_dcp_merge_attn",
+    "qsa_dcp_merge_attn", "qsa_selftest_bounded_wait",
     "qsa_last_error_string", "qsa_status_name", "qsa_abi_version",
 )
 
@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
     L.qsa_sparse_attn_prefill_workspace_size.restype = U
     L.qsa_get_device_status.argtypes = [P, P, I, P]
     L.qsa_get_device_status.restype = I
+    L.qsa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P, P, P]
+    L.qsa_selftest_bounded_wait.restype = I
     L.qsa_index_scores.argtypes = [P, I, P, P, I, I, P, I, I, P, P, I, I, I, P, I, P, P, P]
     L.qsa_topk_groups_workspace_size.argtypes = [I, I, I]
     L.qsa_topk_groups_workspace_size.restype = U
@@ -201,6 +203,15 @@ def qsa_sparse_attn_prefill_workspace_size(T, Hq, Hkv, D, W, kv_dtype=QSA_BF16) 
     if isinstance(kv_dtype, torch.dtype):
         kv_dtype = _dt(torch.empty(0, dtype=kv_dtype))
     return int(lib().qsa_sparse_attn_prefill_workspace_size(T, Hq, Hkv, D, W, kv_dtype))
+
+
+def qsa_selftest_bounded_wait(limit_us, dev_status, report, stream=None):
+    """Run the bounded-wait self-test (a wait on a barrier nothing arrives
+    at, with a limit of limit_us): report is int32 [6] on the device."""
+    if report.numel() < 6 or report.dtype != torch.int32:
+        raise ValueError("report must be int32 with at least 6 elements")
+    _check(lib().qsa_selftest_bounded_wait(int(limit_us), _ptr(dev_status), _ptr(report), _stream(stream)))
+    return report
 
 
 def qsa_get_device_status(dev_status, clear=False, stream=None):

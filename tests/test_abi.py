@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 9
+    assert L.qsa_abi_version() == 10
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -181,6 +181,18 @@ def test_device_status_query_checks_its_pointer(L):
     assert L.qsa_get_device_status(ctypes.c_void_p(0x2002), ctypes.byref(bits), 1, NULL) == 1
     assert "aligned" in _err(L)
     assert bits.value == 7
+
+
+def test_bounded_wait_selftest_validation(L):
+    """The self-test refuses null pointers and limits outside 1 us .. 1 s on
+    the host, before any launch."""
+    ok = ctypes.c_void_p(0x2000)
+    f = L.qsa_selftest_bounded_wait
+    f.argtypes = [ctypes.c_uint32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert f(1000, NULL, ok, NULL) == 1 and "null" in _err(L)
+    assert f(1000, ok, NULL, NULL) == 1
+    assert f(0, ok, ok, NULL) == 1 and "limit_us" in _err(L)
+    assert f(1000001, ok, ok, NULL) == 1 and "limit_us" in _err(L)
 
 
 def test_indexer_write_validation(L):
