@@ -168,6 +168,21 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs a, AttnScale
   const size_t th = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const float* ml = ws_ml + th * splits * 2;
+  // thread -> (float4 column, split group); the first kPre partials of the
+  // thread's group are loaded now, so their L2 latency overlaps the
+  // reductions of the (max, sum) pairs below
+  const float* po = ws_o + th * splits * a.D;
+  const int ncol = a.D / 4;
+  const int ngrp = blockDim.x / ncol;  // >= 1
+  const int col = tid % ncol, grp = tid / ncol;
+  constexpr int kPre = 4;
+  float4 pre[kPre];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) {
+    const int s = grp + u * ngrp;
+    pre[u] = (grp < ngrp && s < splits) ? *reinterpret_cast<const float4*>(po + (size_t)s * a.D + 4 * col)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float M = -INFINITY;
   for (int s = tid; s < splits; s += blockDim.x) M = fmaxf(M, ml[2 * s]);
 #pragma unroll
@@ -193,14 +208,17 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(AttnArgs a, AttnScale
   pdl_launch_dependents();
   __syncthreads();  // fs complete
   const float inv = L > 0.f ? sc.vmul / L : 0.f;
-  const float* po = ws_o + th * splits * a.D;
-  // thread -> (float4 column, split group); the groups' sums meet in shared memory
-  const int ncol = a.D / 4;
-  const int ngrp = blockDim.x / ncol;  // >= 1
-  const int col = tid % ncol, grp = tid / ncol;
+  // the groups' sums meet in shared memory
   float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
   if (grp < ngrp) {
-    int s = grp;
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int s = grp + u * ngrp;
+      const float f = s < splits ? fs[s] : 0.f;
+      O.x = fmaf(pre[u].x, f, O.x); O.y = fmaf(pre[u].y, f, O.y);
+      O.z = fmaf(pre[u].z, f, O.z); O.w = fmaf(pre[u].w, f, O.w);
+    }
+    int s = grp + kPre * ngrp;
     for (; s + 3 * ngrp < splits; s += 4 * ngrp) {  // four loads in flight
       float4 v[4];
       float f[4];
