@@ -265,12 +265,12 @@ QSA_API qsa_status_t qsa_dense_select(const int32_t* q_pos, int T, int threshold
  * sm_scale <= 0.  lse may be NULL.
  * Supported: D in {64, 128, 256}, Hq/Hkv <= 16, q_dt F32 or BF16, kv_dt F32,
  * BF16 or FP8_E4M3, out_dt F32 or BF16.
- * _decode splits every row's tokens across the CTAs of one thread-block
- * cluster per (query, KV head), which merge their partials on chip; only
- * rows too long for one cluster are split over several, whose partials go
- * through qsa_sparse_attn_decode_workspace_size(..., kv_dt) bytes of
- * workspace (0 when none is needed).  _prefill gives each (query, KV head)
- * its own warp and needs no workspace. */
+ * _decode with fewer (query, KV head) rows than SMs (the BF16 / FP8 caches,
+ * D 128 or 256) splits every row's tokens over several CTAs, one per SM;
+ * each CTA leaves its partial (o, max, sum) in the workspace and a second
+ * kernel merges a row's partials: qsa_sparse_attn_decode_workspace_size(...,
+ * kv_dt) bytes (0 when the rows fill the GPU and nothing is split).
+ * _prefill gives each (query, KV head) its own warp and needs no workspace. */
 QSA_API size_t qsa_sparse_attn_decode_workspace_size(int T, int Hq, int Hkv, int D, int W,
                                                      qsa_dtype_t kv_dt);
 QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void* k_pages,
