@@ -196,13 +196,18 @@ QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint
  * Top-K, for group budgets of 512, 1,024 and 2,048, falling back to the exact
  * radix Top-K otherwise).  Same inputs, outputs and result as
  * qsa_topk_groups: the exact top-min(K, c) of every row, ties to the lower
- * group id, ascending, -1 padded.  Per row it guesses a threshold from a
- * strided sample of the row's own scores, verifies by counting the scores
- * that reach it (re-guessing from the sample when the count is too small or
- * too large), and refines with an exact select among the gathered
- * candidates; a row whose guesses fail takes a radix select over the whole
- * row.  path (optional, [T] int32) receives per row: 0 dense (c <= K), 1 the
- * first guess verified, 2 a later guess verified, 3 the whole-row select.
+ * group id, ascending, -1 padded.  Per row it guesses from a strided sample
+ * of the row's own scores where the K-th largest lies, verifies the guess by
+ * exact counts, and refines with an exact select among the candidates the
+ * guess leaves; a row whose guess fails takes a radix select over the whole
+ * row.  Few long rows (under 148 rows of more than 8,192 candidates: decode)
+ * run on one thread-block cluster per row: the guess is a window of key bins
+ * around the sample's rank of the K-th key, the counts above and in it are
+ * exact over the cluster.  Many rows run one CTA per row: the guess is a
+ * threshold, re-guessed from the sample up to twice when its count is too
+ * small or too large.  path (optional, [T] int32) receives per row: 0 dense
+ * (c <= K), 1 the first guess verified, 2 a later guess verified, 3 the
+ * whole-row select.
  * For K outside {512, 1024, 2048} the call runs qsa_topk_groups instead (a
  * message on stderr the first time) and leaves path unwritten. */
 QSA_API qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,

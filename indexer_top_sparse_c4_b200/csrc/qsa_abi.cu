@@ -320,6 +320,13 @@ qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const in
   }
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
+  if (T < 148 && qsa::topk_cluster_size(score_stride) > 1) {
+    // few long rows (decode): the cluster Top-K with the self-sampled guess
+    qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
+    a.gvr = 1;
+    a.path = path;
+    return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups_gvr launch");
+  }
   return cuda_status(qsa::launch_topk_gvr(scores, score_stride, q_pos, T, K, sel, n_sel, path, (cudaStream_t)stream),
                      "qsa_topk_groups_gvr launch");
 }

@@ -224,6 +224,11 @@ struct TopkArgs {
   // optional [T][kPrefixBins] prefix histogram from the scan: read in place of
   // the first cluster passes where a row's total matches, then zeroed
   uint32_t* hist = nullptr;
+  // guess-verify-refine with self-sampling (cluster kernel, no histogram): the
+  // guess is a window of key bins read off a strided sample of the row;
+  // path (optional) gets 0 dense, 1 the guess verified, 3 the cluster passes
+  int gvr = 0;
+  int32_t* path = nullptr;
 };
 int topk_cluster_size(int score_stride);       // 0: unsupported
 cudaError_t launch_topk_groups(const TopkArgs& a, cudaStream_t s);

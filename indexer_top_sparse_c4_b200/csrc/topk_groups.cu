@@ -36,6 +36,13 @@
 //      adds the slots and finds the digit itself.  After two passes the keys
 //      that still match the 16-bit prefix (usually a few dozen) are pushed
 //      into every CTA, which finishes the last two digits locally.
+//    - Guess-verify-refine with self-sampling (no histogram): every CTA reads
+//      the same strided sample of 2,048 of the row's scores and takes, from a
+//      histogram of their top 12 key bits, the window of bins between the
+//      sample ranks n*2048/c -+ (3 sigma + 1).  The keys in the window are the
+//      candidates and the exact counts verify the guess as above; after the
+//      pull, one 256-bin pass over the window finds the exact bin and the
+//      digit passes go on.  A failed guess takes the cluster passes.
 //    - The counts of the CTAs before a CTA come from data every CTA already
 //      holds (the pass tables, or the exchanged counts), so the output needs
 //      no further exchange.
@@ -54,13 +61,16 @@ constexpr int kBins = 256;
 constexpr int kMaxCL = 8;
 
 constexpr int kCandCap = 2048;  // candidates gathered by a cluster (else more cluster passes)
+constexpr int kListCapG = 4096; // self-sampling window path: candidates listed by a cluster
+constexpr int kSampleN = 2048;  // self-sampling guess: scores sampled per row
 constexpr int kRankCap = 512;   // up to this many candidates are ranked directly
 constexpr int kKeptCap = kWarps * kBins;  // kept ids a CTA stages for its coalesced output
 
-struct __align__(16) TopkSmem {
+template <int CAP>
+struct __align__(16) TopkSmemT {
   uint32_t hw[kWarps][kBins];            // per-warp histogram of the current digit
   uint32_t hall[4][kMaxCL][kBins];       // per pass: slot q = CTA q's histogram
-  uint2 cand[kCandCap];                  // (key, id) candidates
+  uint2 cand[CAP];                       // (key, id) candidates
   int wsum[kWarps][kMaxCL];              // block reduction of the per-CTA counts above tau
   int ccnt[2 * kMaxCL];                  // per CTA: candidates above tau, equal to tau
   int wa[kWarps];                        // per-warp scan totals
@@ -68,13 +78,18 @@ struct __align__(16) TopkSmem {
   uint32_t tau;
   // prefix-histogram path: the bin of the n-th largest key (from the
   // histogram), and per source CTA its keys in and above that bin
-  int pbin;
+  int pbin, pbin_lo;                     // the guessed window of 12-bit bins (one bin: equal)
   int scnt[kMaxCL], sgt[kMaxCL];
   uint2 fin[kRankCap];                   // candidates left after the first local digit
   int nfin;
 };
 static_assert(kThreads * 8 == kPrefixBins, "each thread reads 8 bins of the prefix histogram");
-static_assert(sizeof(TopkSmem) % 16 == 0, "the key array after TopkSmem starts on 16 bytes");
+static_assert(kWarps * kBins == kPrefixBins && kSampleN % kThreads == 0 && 4 * kMaxCL >= kWarps,
+              "the sample histogram reuses hw, 8 bins per thread");
+using TopkSmem = TopkSmemT<kCandCap>;   // the histogram / plain paths
+using TopkSmemG = TopkSmemT<kListCapG>; // the self-sampling path
+static_assert(sizeof(TopkSmem) % 16 == 0 && sizeof(TopkSmemG) % 16 == 0,
+              "the key array after the shared struct starts on 16 bytes");
 
 // A thread's KPT keys.  RegKeys: in registers (loops over them fully
 // unrolled).  SmemKeys: in shared memory, key j of thread i at [j][i], so
@@ -196,7 +211,10 @@ __device__ __forceinline__ void dense_row(const TopkArgs& a, const Row& r, int t
       if (total > a.W) flag(a.status, QSA_DEV_ROW_RANGE);
     }
   }
-  if (rank == 0 && tid == 0) a.n_sel[t] = r.n;
+  if (rank == 0 && tid == 0) {
+    a.n_sel[t] = r.n;
+    if (a.path) a.path[t] = 0;
+  }
 }
 
 // The thread's KPT consecutive candidates from `first`, as keys (0 past c).
@@ -226,8 +244,8 @@ __device__ __forceinline__ void load_keys(Keys& keys, const float* row, int firs
 // all KPT.  The ids are staged in shared memory (the per-warp histograms,
 // whose last use came before the block scan that gave the positions) and
 // written with coalesced stores.
-template <int KPT, bool MASKED, typename Keys>
-__device__ __forceinline__ void emit_kept(TopkSmem& sm, const Keys& keys, uint64_t above_mask, uint64_t cand_mask,
+template <int KPT, bool MASKED, typename Keys, typename SM>
+__device__ __forceinline__ void emit_kept(SM& sm, const Keys& keys, uint64_t above_mask, uint64_t cand_mask,
                                           int first, uint32_t tau, int gt, int gt_before, int eq_before, int cta_gt,
                                           int cta_eq, int rem, int off, const Row& r, int tvec) {
   constexpr int U = Keys::kUnroll;
@@ -381,15 +399,17 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
 }
 
 // ---- few long rows: one cluster per row, keys in shared memory ------------------
-template <int CL, int KPT>
+template <int CL, int KPT, bool GVR>
 __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, int vec, int tvec) {
   static_assert(CL > 1, "one-CTA rows use topk_row_kernel");
   static_assert(KPT <= 64, "key masks are 64 bits");
+  using SMT = TopkSmemT<GVR ? kListCapG : kCandCap>;
   constexpr int U = SmemKeys<KPT>::kUnroll;
-  constexpr int kSeg = kCandCap / CL;           // histogram path: list capacity per CTA
-  constexpr int kSlots = kCandCap / kThreads;   // histogram path: list entries per thread
+  constexpr int kCap = GVR ? kListCapG : kCandCap;
+  constexpr int kSeg = kCap / CL;           // bin / window path: list capacity per CTA
+  constexpr int kSlots = kCap / kThreads;   // bin / window path: list entries per thread
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  SMT& sm = *reinterpret_cast<SMT*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
@@ -421,15 +441,26 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     }
   }
   uint4 hv0 = make_uint4(0u, 0u, 0u, 0u), hv1 = hv0;
-  if (r.hrow) {
+  if (!GVR && r.hrow) {
     hv0 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 8 - 8 * tid));
     hv1 = __ldcg(reinterpret_cast<const uint4*>(r.hrow + kPrefixBins - 4 - 8 * tid));
+  }
+  // self-sampling guess: sample i of ns is candidate i * c / ns -- the same
+  // positions in every CTA of the cluster (every candidate when c <= kSampleN)
+  const int ns = c < kSampleN ? c : kSampleN;
+  float smp[kSampleN / kThreads];
+  if constexpr (GVR) {
+#pragma unroll
+    for (int k = 0; k < kSampleN / kThreads; ++k) {
+      const int i = tid + k * kThreads;
+      smp[k] = i < ns ? __ldg(row + (int)(((long long)i * c) / ns)) : 0.f;
+    }
   }
 
   // ---- the bin of the n-th largest key, from the histogram
   bool hist_ok = false;  // (the same in every CTA: they read the same histogram)
   uint32_t pb = 0;
-  if (r.hrow) {
+  if (!GVR && r.hrow) {
     const uint32_t hb[8] = {hv1.w, hv1.z, hv1.y, hv1.x, hv0.w, hv0.z, hv0.y, hv0.x};
     int hs = 0;
 #pragma unroll
@@ -451,9 +482,55 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     }
   }
 
-  // ---- keys into shared memory; on the histogram path, which of them lie
-  // above the bin (kept for sure) and in it (the candidates)
-  SmemKeys<KPT> keys{reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkSmem)) + tid};
+  uint32_t pb_lo = pb;  // the window of bins [pb_lo, pb] (one bin on the histogram path)
+  if constexpr (GVR) {
+    // ---- guess: a histogram of the sample's top 12 key bits (in hw, which
+    // only this CTA writes: the cluster passes write the other CTAs' hall, and
+    // a peer may start them before this CTA is done here); the window spans
+    // the bins of the sample ranks n ns / c -+ (3 sigma + 1): the n-th largest key of the row
+    // lies between them unless the sample is far off, which the exact counts
+    // below catch
+    uint32_t* sh = &sm.hw[0][0];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) sh[8 * tid + j] = 0u;
+    if (tid == 0) {
+      sm.pbin = kPrefixBins - 1;
+      sm.pbin_lo = 0;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kSampleN / kThreads; ++k)
+      if (tid + k * kThreads < ns) atomicAdd(&sh[order_key(smp[k]) >> kPrefixShift], 1u);
+    __syncthreads();
+    uint32_t hb[8];
+    int hs = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      hb[j] = sh[kPrefixBins - 1 - 8 * tid - j];
+      hs += (int)hb[j];
+    }
+    int htotal;
+    const int hbefore = block_exclusive_scan(hs, sm.wa, htotal);
+    const float e = (float)n * (float)ns / (float)c, sd = sqrtf(e);
+    const int r_hi = max(1, (int)floorf(e - 3.f * sd - 1.f));
+    const int r_lo = min(ns, (int)ceilf(e + 3.f * sd + 1.f));
+    int ab = hbefore;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int b = kPrefixBins - 1 - 8 * tid - j;
+      if (ab < r_hi && ab + (int)hb[j] >= r_hi) sm.pbin = b;
+      if (ab < r_lo && ab + (int)hb[j] >= r_lo) sm.pbin_lo = b;
+      ab += (int)hb[j];
+    }
+    __syncthreads();
+    pb = (uint32_t)sm.pbin;
+    pb_lo = (uint32_t)sm.pbin_lo;
+    hist_ok = pb - pb_lo < (uint32_t)kBins;  // the exact bin is then found with one 256-bin pass
+  }
+
+  // ---- keys into shared memory; on the histogram (or window) path, which of
+  // them lie above the bin (kept for sure) and in it (the candidates)
+  SmemKeys<KPT> keys{reinterpret_cast<uint32_t*>(smem_raw + sizeof(SMT)) + tid};
   uint64_t above_mask = 0, cand_mask = 0;
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
@@ -461,7 +538,11 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     const uint32_t k = valid ? order_key(sc[j]) : 0u;
     keys.set(j, k);
     if (valid && (k >> kPrefixShift) > pb) above_mask |= 1ull << j;
-    if (valid && (k >> kPrefixShift) == pb) cand_mask |= 1ull << j;
+    if constexpr (GVR) {
+      if (valid && (k >> kPrefixShift) <= pb && (k >> kPrefixShift) >= pb_lo) cand_mask |= 1ull << j;
+    } else {
+      if (valid && (k >> kPrefixShift) == pb) cand_mask |= 1ull << j;
+    }
   }
 
   uint32_t prefix = 0;
@@ -506,7 +587,6 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     if (!over && above_bin < n && above_bin + in_bin >= n) {
       mode = 2;
       need = n - above_bin;
-      prefix = pb << kPrefixShift;
       // ---- pull every CTA's list into registers (independent DSMEM loads):
       // slot s of thread tid is entry (tid + s*kThreads) % kSeg of CTA
       // (tid + s*kThreads) / kSeg; then release the lists for their CTAs' exit
@@ -521,8 +601,37 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
           valid |= 1u << s;
         }
       }
-      zero_hist_share<CL>(r.hrow, rank);
+      if (r.hrow) zero_hist_share<CL>(r.hrow, rank);
       asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+      const uint32_t valid_all = valid;  // every listed candidate (the per-CTA counts below)
+      if (GVR && pb != pb_lo) {
+        // ---- the window: the exact 12-bit bin of the need-th largest among
+        // its candidates; only those in that bin go on to the digit passes.
+        // The candidates crowd into a few bins: per-warp histograms (in hall,
+        // which no peer writes on this path) keep the atomics apart
+        uint32_t* const hflat = &sm.hall[0][0][0];   // [kWarps][kBins] of the [4][kMaxCL][kBins] array
+        uint32_t* wh = hflat + warp * kBins;
+#pragma unroll
+        for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s)
+          if ((valid >> s) & 1u) atomicAdd(&wh[(ck[s].x >> kPrefixShift) - pb_lo], 1u);
+        __syncthreads();
+        if (tid < kBins) {
+          int h = 0;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) h += (int)hflat[w * kBins + kBins - 1 - tid];
+          find_bin(h, need, kBins - 1 - tid, &sm.bin[3], &sm.above[3], sm.wa);
+        }
+        __syncthreads();
+        pb = pb_lo + (uint32_t)sm.bin[3];
+        need -= sm.above[3];
+#pragma unroll
+        for (int s = 0; s < kSlots; ++s)
+          if ((ck[s].x >> kPrefixShift) != pb) valid &= ~(1u << s);
+      }
+      prefix = pb << kPrefixShift;
       // ---- key bits 12..19 over the candidates
 #pragma unroll
       for (int s = 0; s < kSlots; ++s)
@@ -578,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
       // per source CTA: candidates above and equal to tau
 #pragma unroll
       for (int s = 0; s < kSlots; ++s) {
-        if ((valid >> s) & 1u) {
+        if ((valid_all >> s) & 1u) {
           const int q = (tid + s * kThreads) / kSeg;
           if (ck[s].x > prefix) atomicAdd(&sm.ccnt[q], 1);
           else if (ck[s].x == prefix) atomicAdd(&sm.ccnt[kMaxCL + q], 1);
@@ -789,12 +898,14 @@ __global__ void __launch_bounds__(kThreads, 1) topk_cluster_kernel(TopkArgs a, i
     emit_kept<KPT, false>(sm, keys, 0, 0, first, tau, gt, before & 0xffff, before >> 16, both & 0xffff,
                           both >> 16, rem, off, r, tvec);
   if (rank == 0) write_tail(a, r, t);
+  if (GVR && rank == 0 && tid == 0 && a.path) a.path[t] = mode == 2 ? 1 : 3;
   // the other CTAs read this CTA's candidate list: stay until they have
   if (mode == 2) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <int CL, int KPT>
 cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
+  static_assert(CL >= 1, "cluster size");
   const int vec = (a.score_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
   const int tvec = a.tok && a.W % 4 == 0 && (reinterpret_cast<uintptr_t>(a.tok) & 15u) == 0;
   if constexpr (CL == 1) {
@@ -804,11 +915,14 @@ cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     return launch_k(kern, dim3(1, a.T), dim3(kThreads), smem, s, 1, a, vec, tvec);
   } else {
-    const size_t smem = sizeof(TopkSmem) + (size_t)KPT * kThreads * sizeof(uint32_t);
-    auto kern = topk_cluster_kernel<CL, KPT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec, tvec);
+    auto go = [&](auto kern, size_t base) -> cudaError_t {
+      const size_t smem = base + (size_t)KPT * kThreads * sizeof(uint32_t);
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      return launch_k(kern, dim3(CL, a.T), dim3(kThreads), smem, s, CL, a, vec, tvec);
+    };
+    return a.gvr ? go(topk_cluster_kernel<CL, KPT, true>, sizeof(TopkSmemG))
+                 : go(topk_cluster_kernel<CL, KPT, false>, sizeof(TopkSmem));
   }
 }
 

@@ -3,6 +3,11 @@
 // enable_heuristic_topk: the GVR Top-K for group budgets of 512, 1,024 and
 // 2,048, with the exact radix Top-K as the fallback).
 //
+// This kernel serves calls with many rows (one CTA each).  Few long rows
+// (decode) run on a thread-block cluster per row instead: the cluster Top-K of
+// topk_groups.cu in its self-sampling mode, whose guess is a window of key
+// bins read off a strided sample, verified by exact cluster-wide counts.
+//
 // One CTA of 1024 threads per row; the result is the exact top-K, ties to
 // the lower group id, ascending:
 //  * guess: S = 4,096 scores sampled at even strides over the row's c

@@ -95,6 +95,27 @@ def test_gvr_falls_back_on_equal_scores(q, oracle):
     assert np.array_equal(host(sel), ref)
 
 
+@pytest.mark.parametrize("K", [512, 2048])
+def test_gvr_guess_missed_by_the_sample_is_caught(q, oracle, K):
+    """Decode rows whose largest scores sit only at ids the strided sample
+    never reads (i * c // 2048 is 31 mod 32 for c = 65,535): the guessed
+    window lies far below the true K-th score, the exact counts reject it,
+    and the row takes the cluster passes -- with the exact result."""
+    T, c = 2, 65535
+    g = torch.Generator(device="cpu").manual_seed(17)
+    scores = torch.randn((T, c + 1), generator=g)
+    hidden = torch.arange(7, c, 16)[: K + 100]
+    scores[:, hidden] = 50.0 + torch.rand((T, hidden.numel()), generator=g)
+    scores = scores.cuda()
+    q_pos = torch.full((T,), 4 * c + 3, dtype=torch.int32, device="cuda")
+    sel, n_sel, path = _gvr(q, scores, q_pos, K)
+    assert host(path).tolist() == [3, 3]
+    rs, rn = _radix(q, scores, q_pos, K)
+    assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
+    ref, nref = oracle.topk_groups(host(scores), host(q_pos), K)
+    assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref)
+
+
 def test_gvr_other_budgets_use_the_radix_top_k(q):
     w = wl.b1_16k(device="cuda", K=300)
     st = QSAStep(w)
