@@ -116,6 +116,27 @@ def test_gvr_guess_missed_by_the_sample_is_caught(q, oracle, K):
     assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref)
 
 
+@pytest.mark.parametrize("c, stride", [(131071, 131072), (100000, 100003), (250001, 262144)])
+def test_gvr_cluster_rows_beyond_262k_tokens_and_odd_strides(q, oracle, c, stride):
+    """Longer rows than the 262,144-token workload (32 and 64 keys per
+    thread in the cluster) and a row stride that is not a multiple of 4
+    (scalar loads): the self-sampled guess, against the radix Top-K and the
+    oracle, at the three budgets."""
+    T = 3
+    g = torch.Generator(device="cpu").manual_seed(c % 1000)
+    scores = torch.randn((T, stride), generator=g)
+    scores[1] = torch.round(scores[1] * 4) / 4          # a row of many ties
+    scores = scores.cuda()
+    q_pos = torch.tensor([4 * c + 3, 4 * c, 4 * c + 1], dtype=torch.int32, device="cuda")
+    for K in (512, 1024, 2048):
+        sel, n_sel, path = _gvr(q, scores, q_pos, K)
+        rs, rn = _radix(q, scores, q_pos, K)
+        assert torch.equal(sel, rs) and torch.equal(n_sel, rn), K
+        ref, nref = oracle.topk_groups(host(scores), host(q_pos), K)
+        assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref), K
+        assert set(host(path).tolist()) <= {1, 3}
+
+
 def test_gvr_other_budgets_use_the_radix_top_k(q):
     w = wl.b1_16k(device="cuda", K=300)
     st = QSAStep(w)
