@@ -33,12 +33,6 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-// two FP8-E4M3 codes (low byte first) -> f16x2, exact
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-  return (uint32_t)h.x | ((uint32_t)h.y << 16);
-}
-
 // four FP8-E4M3 codes (byte 0 first) -> two f16x2: codes 0, 1 in `lo`,
 // codes 2, 3 in `hi`, exact; the word's halves feed the conversion directly
 __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, uint32_t& hi) {
@@ -73,7 +67,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 __device__ __forceinline__ uint4 lds16(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
-__device__ __forceinline__ uint4 ldg16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
 // Tile geometry for one KV storage type and head dim.
 template <bool FP8, int D>
@@ -88,16 +81,7 @@ struct Geo {
   static constexpr int MT = D / 16;            // PV m-tiles (output dims / 16)
   static constexpr int MTJ = CH / 2;           // m-tiles fed by one V chunk
   static constexpr int ROWB = D * EB;          // bytes of one K (or V) row of one KV head
-  static constexpr int NW = 4;                 // warps per CTA: a round is one tile per warp
-  static constexpr int ROUND = 16 * NW;        // tokens per round
-  static constexpr int STAGE = ROUND * 2 * ROWB;  // K rows, then V rows
-  // FP8 rows are half the size: three 32 KiB stages keep a CTA near 104 KiB of
-  // shared memory, two CTAs per SM, so clusters of 8 all fit at once; BF16
-  // keeps two 64 KiB stages at one CTA per SM
-  static constexpr int NSTAGE = FP8 ? 3 : 2;
-  static constexpr int OFFCAP = 1024;          // row offsets looked up per batch
   static_assert(NCH % 8 == 0, "V chunks must split over 8 lanes");
-  static_assert(OFFCAP % ROUND == 0, "a batch holds whole rounds");
 };
 
 // Byte offset of the K/V row (this KV head) of token slot `i` of the list, or

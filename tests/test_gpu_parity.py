@@ -403,20 +403,22 @@ def test_tensor_parallel_heads(kv):
 
 
 GATHER_PLANS = [  # (B, ctx, (Hq, Hkv), K, kv): decode plans of the gather kernel
-    (1, 16384, (16, 2), 2048, "bf16"),    # 2 rows of 8,196 slots: 5 clusters of 15 + combine
-    (2, 65536, (16, 2), 4096, "fp8"),     # 4 rows of 16,388 slots: 5 clusters of 15 + combine
-    (4, 16384, (12, 1), 1024, "fp8"),     # 12 heads per KV head (two warps per slot), 3 clusters
-    (3, 16384, (6, 1), 512, "bf16"),      # 6 heads per KV head, one cluster of 16 per row
-    (40, 8192, (16, 2), 512, "fp8"),      # 80 rows: clusters of 4
-    (1, 262144, (3, 1), 8192, "fp8"),     # 32,772 slots: 33 chunks of 1,024 (the table's capacity)
+    (1, 16384, (16, 2), 2048, "bf16"),    # 2 rows x 74 chunks of 112 slots (four two-stage BF16 slots), combine
+    (2, 65536, (16, 2), 4096, "fp8"),     # 4 rows x 37 chunks of 448 slots, combine
+    (4, 16384, (12, 1), 1024, "fp8"),     # 12 heads per KV head: two warps per slot, 37 chunks per row
+    (3, 16384, (6, 1), 512, "bf16"),      # 6 heads per KV head; 33 chunks per row (one tile per slot)
+    (40, 8192, (16, 2), 512, "fp8"),      # 80 rows x 3 chunks of 688 (240 CTAs, two waves), combine
+    (40, 8192, (16, 2), 128, "fp8"),      # 80 rows of 516 slots: one chunk per row, the output written directly
+    (8, 65536, (16, 2), 4096, "fp8"),     # 16 rows x 17 chunks of 976 (the row-index table's 1,024), two waves
 ]
 
 
 @pytest.mark.parametrize("case", GATHER_PLANS, ids=lambda c: f"b{c[0]}_c{c[1]}_h{c[2][0]}x{c[2][1]}_k{c[3]}_{c[4]}")
 def test_decode_gather_plans(oracle, case):
-    """The decode attention's plans: one cluster per row, several clusters per
-    row merged by the combine kernel, two warps per slot, chunks limited by
-    the row-index table; every row against the oracle."""
+    """The decode attention's plans: rows split into many chunks merged by
+    the combine kernel, one chunk per row written directly, two warps per
+    slot, BF16 and FP8 stage sizes, chunks limited by the row-index table;
+    every row against the oracle."""
     B, ctx, (Hq, Hkv), K, kv = case
     w = wl.make(f"gather_{B}_{ctx}", B=B, ctx=ctx, Hq=Hq, Hkv=Hkv, D=256, H_I=4, D_I=128, K=K, kv_dtype=kv,
                 q_dtype="bf16", dist="peaked", seed=B + K, device="cuda")
