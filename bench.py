@@ -67,8 +67,9 @@ def profiled_traffic(context):
 
 
 def algorithmic_bytes(w, n_tok_total):
-    """spec byte count of one step: every candidate group's compressed
-    key, plus K and V rows of every selected token for every KV head."""
+    """Algorithmic bytes of one step (the headline metric's definition):
+    every candidate group's compressed key, plus the K and V rows of every
+    selected token for every KV head."""
     kv_elem = {"fp8": 1, "bf16": 2, "f32": 4}[w.kv_dtype]
     idx_elem = w.k_idx_pages.element_size()
     groups = int((w.q_pos // 4).sum().item())

@@ -5,8 +5,9 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-# attention tolerances against the FP64 oracle (max-abs, mean-abs as the
-# spec states them; rel-L2 as the Ascend operator tests use)
+# attention tolerances against the FP64 oracle (max-abs 2e-2 and mean-abs
+# 2e-3 for BF16 / FP8 KV, the target stated for this path; rel-L2 as the
+# Ascend article's operator tests use)
 ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 2e-3
 ATTN_REL_L2 = 8e-3
