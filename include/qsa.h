@@ -288,6 +288,31 @@ QSA_API qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, con
                                     void* workspace, size_t workspace_bytes,
                                     uint32_t* dev_status, qsa_stream_t stream);
 
+/* Stages 3 and 4 in one call for decode: exactly
+ *   qsa_expand_select(sel, n_sel, K, q_pos, capture_pos, T, tok, n_tok, W)
+ *   qsa_sparse_attn_decode(..., tok, n_tok, W, ...)
+ * with the same out / lse and status bits, without the token lists in
+ * between: the decode kernel that spreads few rows over every SM (BF16 / FP8
+ * caches, D 128 or 256) lists each chunk's tokens from the selection itself
+ * (4 per kept group, then 4*c(p0) .. p, cut at W).  For other shapes the
+ * call writes the lists into its workspace first and runs the regular
+ * decode.  capture_pos may be NULL (no MTP reuse).  W >= 4*K + 4 (+4 per
+ * group completed since the capture).  Workspace:
+ * qsa_sparse_attn_decode_sel_workspace_size(...) bytes, 16-byte aligned
+ * (0: none needed); pointers as for the two calls it replaces. */
+QSA_API size_t qsa_sparse_attn_decode_sel_workspace_size(int T, int Hq, int Hkv, int D, int W,
+                                                         qsa_dtype_t kv_dt);
+QSA_API qsa_status_t qsa_sparse_attn_decode_sel(const void* q, qsa_dtype_t q_dt, const void* k_pages,
+                                                const void* v_pages, qsa_dtype_t kv_dt, float k_scale,
+                                                float v_scale, int num_pages, const int32_t* page_table,
+                                                int pt_rows, int pt_stride, const int32_t* q_req,
+                                                const int32_t* sel, const int32_t* n_sel, int K,
+                                                const int32_t* q_pos, const int32_t* capture_pos, int W, int T,
+                                                int Hq, int Hkv, int D, float sm_scale, void* out,
+                                                qsa_dtype_t out_dt, float* lse, void* workspace,
+                                                size_t workspace_bytes, uint32_t* dev_status,
+                                                qsa_stream_t stream);
+
 /* Workspace of qsa_sparse_attn_prefill: 0 bytes (each (query, KV head) row is
  * finished by the warps that stream it). */
 QSA_API size_t qsa_sparse_attn_prefill_workspace_size(int T, int Hq, int Hkv, int D, int W,
@@ -429,7 +454,7 @@ QSA_API const char* qsa_status_name(qsa_status_t s);
  * and a workspace query for every stage; 6: qsa_indexer_project and
  * qsa_compress_keys; 7: the sequence-sharded decode calls qsa_dcp_*; 8:
  * qsa_topk_groups_gvr; 9: qsa_seq_len_threshold and qsa_dense_select; 10:
- * qsa_selftest_bounded_wait). */
+ * qsa_selftest_bounded_wait; 11: qsa_sparse_attn_decode_sel). */
 QSA_API int qsa_abi_version(void);
 
 #ifdef __cplusplus

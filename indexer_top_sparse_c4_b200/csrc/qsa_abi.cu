@@ -97,7 +97,7 @@ const char* qsa_status_name(qsa_status_t s) {
   return "QSA_ERR_UNKNOWN";
 }
 
-int qsa_abi_version(void) { return 10; }
+int qsa_abi_version(void) { return 11; }
 
 size_t qsa_index_scores_workspace_size(int T, int H_I, int D_I, int score_stride) {
   (void)T; (void)H_I; (void)D_I; (void)score_stride;
@@ -409,6 +409,67 @@ qsa_status_t qsa_sparse_attn_decode(const void* q, qsa_dtype_t q_dt, const void*
                   dev_status};
   return cuda_status(qsa::launch_sparse_attn(a, plan, workspace, (cudaStream_t)stream, true),
                      "qsa_sparse_attn_decode launch");
+}
+
+namespace {
+size_t align16z(size_t n) { return (n + 15) & ~(size_t)15; }
+// The fused call's workspace: the decode plan's partials, plus -- for plans
+// other than the gather kernel's -- the token lists the expansion writes first.
+size_t decode_sel_ws(const qsa::DecodePlan& plan, int T, int Hq, int D, int W) {
+  const size_t attn = qsa::attn_decode_ws_bytes(T, Hq, D, plan.s);
+  if (plan.gather) return attn;
+  return align16z(attn) + align16z((size_t)T * W * sizeof(int32_t)) + align16z((size_t)T * sizeof(int32_t));
+}
+}  // namespace
+
+size_t qsa_sparse_attn_decode_sel_workspace_size(int T, int Hq, int Hkv, int D, int W, qsa_dtype_t kv_dt) {
+  if (T <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || W <= 0) return 0;
+  return decode_sel_ws(qsa::attn_decode_plan(T, Hq, Hkv, D, W, kv_dt), T, Hq, D, W);
+}
+
+qsa_status_t qsa_sparse_attn_decode_sel(const void* q, qsa_dtype_t q_dt, const void* k_pages, const void* v_pages,
+                                        qsa_dtype_t kv_dt, float k_scale, float v_scale, int num_pages,
+                                        const int32_t* page_table, int pt_rows, int pt_stride,
+                                        const int32_t* q_req, const int32_t* sel, const int32_t* n_sel, int K,
+                                        const int32_t* q_pos, const int32_t* capture_pos, int W, int T, int Hq,
+                                        int Hkv, int D, float sm_scale, void* out, qsa_dtype_t out_dt, float* lse,
+                                        void* workspace, size_t workspace_bytes, uint32_t* dev_status,
+                                        qsa_stream_t stream) {
+  REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
+  REQUIRE(W >= 4 * K + 4, "W must be >= 4*K + 4 = %d (got %d)", 4 * K + 4, W);
+  // the selection stands in for the token lists in the shared checks
+  qsa_status_t st = check_attn(q, q_dt, k_pages, v_pages, kv_dt, num_pages, page_table, pt_rows, pt_stride, sel,
+                               n_sel, W, T, Hq, Hkv, D, out, out_dt, k_scale, v_scale);
+  if (st != QSA_OK || T == 0) return st;
+  REQUIRE(q_pos != nullptr, "null pointer argument");
+  const qsa::DecodePlan plan = qsa::attn_decode_plan(T, Hq, Hkv, D, W, kv_dt);
+  const size_t need = decode_sel_ws(plan, T, Hq, D, W);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    return fail(QSA_ERR_WORKSPACE, "decode needs %zu bytes of 16-byte-aligned workspace (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  qsa::AttnArgs a{q, q_dt, k_pages, v_pages, kv_dt, k_scale, v_scale, num_pages, page_table,
+                  pt_rows, pt_stride, q_req, nullptr, nullptr, W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse,
+                  dev_status};
+  const cudaStream_t s = (cudaStream_t)stream;
+  if (plan.gather) {  // the gather kernel lists each chunk's tokens itself
+    a.sel = sel;
+    a.n_sel = n_sel;
+    a.K = K;
+    a.q_pos = q_pos;
+    a.capture_pos = capture_pos;
+    return cuda_status(qsa::launch_sparse_attn(a, plan, workspace, s, true), "qsa_sparse_attn_decode_sel launch");
+  }
+  // other plans: stage 3 into the workspace, then the decode attention
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  int32_t* tok = reinterpret_cast<int32_t*>(base + align16z(qsa::attn_decode_ws_bytes(T, Hq, D, plan.s)));
+  int32_t* n_tok = reinterpret_cast<int32_t*>(reinterpret_cast<unsigned char*>(tok) +
+                                              align16z((size_t)T * W * sizeof(int32_t)));
+  qsa::ExpandArgs e{sel, n_sel, K, q_pos, capture_pos, T, tok, n_tok, W, dev_status};
+  st = cuda_status(qsa::launch_expand_select(e, s), "qsa_sparse_attn_decode_sel launch");
+  if (st != QSA_OK) return st;
+  a.tok = tok;
+  a.n_tok = n_tok;
+  return cuda_status(qsa::launch_sparse_attn(a, plan, workspace, s, true), "qsa_sparse_attn_decode_sel launch");
 }
 
 qsa_status_t qsa_sparse_attn_prefill(const void* q, qsa_dtype_t q_dt, const void* k_pages,

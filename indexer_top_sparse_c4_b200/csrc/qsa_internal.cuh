@@ -246,6 +246,12 @@ struct AttnArgs {
   float k_scale, v_scale; int num_pages; const int32_t* page_table; int pt_rows, pt_stride;
   const int32_t* q_req; const int32_t* tok; const int32_t* n_tok; int W, T, Hq, Hkv, D;
   float sm_scale; void* out; qsa_dtype_t out_dt; float* lse; uint32_t* status;
+  // selection mode (gather kernel only; tok / n_tok unused): each row's token
+  // slots follow from the kept groups as stage 3 would list them -- 4 per
+  // kept group of sel [T, K] (n_sel of them), then 4*c(p0) .. p with p0 the
+  // capture position (or p) -- cut at W
+  const int32_t* sel = nullptr; const int32_t* n_sel = nullptr; int K = 0;
+  const int32_t* q_pos = nullptr; const int32_t* capture_pos = nullptr;
 };
 // Plan of the decode kernel that spreads each (query, KV head) row over S
 // CTAs of C token slots each; with S > 1 the combine kernel merges the S

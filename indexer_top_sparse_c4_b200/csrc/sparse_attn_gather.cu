@@ -124,15 +124,46 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
   pdl_wait();
   // ---- the chunk's cache rows: token id -> page -> row index (-1: skipped).
   // The ids, the row's length and its request are loaded together.
-  const int32_t* trow = a.tok + (size_t)t * a.W;
   int r = a.q_req ? __ldg(a.q_req + t) : t;
-  int nt = __ldg(a.n_tok + t);
   constexpr int IPT = (kGaMaxChunk + NTHR - 1) / NTHR;  // ids per thread at most
   int jv[IPT];
+  int nt;
+  if (a.sel) {
+    // selection mode: slot i of the row is token 4 g + i % 4 of kept group
+    // g = sel[i / 4] while i < 4 n_sel, then 4 c(p0) + (i - 4 n_sel) up to p
+    const int p = __ldg(a.q_pos + t);
+    int p0 = a.capture_pos ? __ldg(a.capture_pos + t) : p;
+    p0 = p0 > p ? p : p0;
+    const int c0 = p0 >= 0 ? p0 / kGroupTokens : 0;
+    int ns = __ldg(a.n_sel + t);
+    ns = ns < 0 ? 0 : (ns > a.K ? a.K : ns);
+    const int head = kGroupTokens * ns, total = head + (p >= 0 ? p - kGroupTokens * c0 + 1 : 0);
+    nt = total < a.W ? total : a.W;
+    if (total > a.W && s == 0 && kvh == 0 && tid == 0) flag(a.status, QSA_DEV_ROW_RANGE);
+    const int32_t* srow = a.sel + (size_t)t * a.K;
 #pragma unroll
-  for (int k = 0; k < IPT; ++k) {
-    const int i = tid + k * NTHR;
-    jv[k] = (i < C && cbeg + i < a.W) ? __ldg(trow + cbeg + i) : -1;
+    for (int k = 0; k < IPT; ++k) {
+      const int i = tid + k * NTHR, ks = cbeg + i;
+      int v = -1;
+      if (i < C && ks < nt) {
+        if (ks < head) {
+          const int g = __ldg(srow + ks / kGroupTokens);
+          if (g >= 0 && g < c0) v = kGroupTokens * g + ks % kGroupTokens;
+          else if (ks % kGroupTokens == 0 && kvh == 0) flag(a.status, QSA_DEV_BAD_GROUP);
+        } else {
+          v = kGroupTokens * c0 + (ks - head);
+        }
+      }
+      jv[k] = v;
+    }
+  } else {
+    const int32_t* trow = a.tok + (size_t)t * a.W;
+    nt = __ldg(a.n_tok + t);
+#pragma unroll
+    for (int k = 0; k < IPT; ++k) {
+      const int i = tid + k * NTHR;
+      jv[k] = (i < C && cbeg + i < a.W) ? __ldg(trow + cbeg + i) : -1;
+    }
   }
   nt = nt < 0 ? 0 : (nt > a.W ? a.W : nt);
   if (r < 0 || r >= a.pt_rows) {

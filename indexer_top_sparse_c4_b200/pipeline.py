@@ -170,9 +170,12 @@ class QSADraftLoop:
 
     Draft step i has one row per capture row (the same request), its own
     attention query (seeded, the capture query's dtype and shape) and its own
-    token lists and output.  Plumbing only: every stage is a libqsa call."""
+    output.  fused (default): each draft step is one qsa_sparse_attn_decode_sel
+    call (stages 3 and 4 together, no token lists); otherwise the expansion
+    writes the draft's token lists and qsa_sparse_attn_decode reads them.
+    Plumbing only: every stage is a libqsa call."""
 
-    def __init__(self, w: Workload, drafts: int = 2, seed: int = 1):
+    def __init__(self, w: Workload, drafts: int = 2, seed: int = 1, fused: bool = True):
         if w.capture_pos is not None:
             raise ValueError("the capture workload is a plain decode workload")
         self.w = w
@@ -190,12 +193,21 @@ class QSADraftLoop:
         self.n_tok = [torch.empty((T,), dtype=torch.int32, device=dev) for _ in range(drafts)]
         self.out = [torch.empty_like(self.capture.out) for _ in range(drafts)]
         self.lse = [torch.empty_like(self.capture.lse) for _ in range(drafts)]
-        ws = qsa.qsa_sparse_attn_decode_workspace_size(T, w.Hq, w.Hkv, w.D, self.W, w.k_pages.dtype)
+        self.fused = fused
+        size = qsa.qsa_sparse_attn_decode_sel_workspace_size if fused else qsa.qsa_sparse_attn_decode_workspace_size
+        ws = size(T, w.Hq, w.Hkv, w.D, self.W, w.k_pages.dtype)
         self.ws = torch.empty((max(ws, 16),), dtype=torch.uint8, device=dev)
         self.status = self.capture.status
 
     def draft_step(self, i: int, stream=None, sm_scale=0.0):
         w, cap = self.w, self.capture
+        if self.fused:
+            qsa.qsa_sparse_attn_decode_sel(self.q[i], w.k_pages, w.v_pages, w.page_table, cap.sel, cap.n_sel,
+                                           self.pos[i], self.W, self.out[i], workspace=self.ws,
+                                           capture_pos=w.q_pos, k_scale=w.k_scale, v_scale=w.v_scale,
+                                           q_req=w.q_req, sm_scale=sm_scale, lse=self.lse[i],
+                                           dev_status=self.status, stream=stream)
+            return
         qsa.qsa_expand_select(cap.sel, cap.n_sel, self.pos[i], self.tok[i], self.n_tok[i],
                               capture_pos=w.q_pos, dev_status=self.status, stream=stream)
         qsa.qsa_sparse_attn_decode(self.q[i], w.k_pages, w.v_pages, w.page_table, self.tok[i],

@@ -31,6 +31,7 @@ ENTRY_POINTS = (
     "qsa_topk_groups", "qsa_topk_groups_gvr", "qsa_expand_select_workspace_size", "qsa_expand_select", "qsa_topk_expand",
     "qsa_seq_len_threshold", "qsa_dense_select",
     "qsa_sparse_attn_decode_workspace_size", "qsa_sparse_attn_decode",
+    "qsa_sparse_attn_decode_sel_workspace_size", "qsa_sparse_attn_decode_sel",
     "qsa_sparse_attn_prefill_workspace_size", "qsa_sparse_attn_prefill", "qsa_get_device_status",
     "qsa_dcp_shard_positions", "qsa_dcp_candidates", "qsa_dcp_merge_topk", "qsa_dcp_expand",
     "qsa_dcp_merge_attn", "qsa_selftest_bounded_wait",
@@ -101,6 +102,11 @@ def lib() -> ctypes.CDLL:
                                          F, P, I, P, P, U, P, P]
     L.qsa_sparse_attn_prefill.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, I, I, I, I,
                                           F, P, I, P, P, P]
+    L.qsa_sparse_attn_decode_sel_workspace_size.argtypes = [I, I, I, I, I, I]
+    L.qsa_sparse_attn_decode_sel_workspace_size.restype = U
+    L.qsa_sparse_attn_decode_sel.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, P, P, I, I, I, I, I,
+                                             F, P, I, P, P, U, P, P]
+    L.qsa_sparse_attn_decode_sel.restype = I
     for name in ("qsa_index_scores", "qsa_topk_groups", "qsa_expand_select", "qsa_topk_expand",
                  "qsa_sparse_attn_decode", "qsa_sparse_attn_prefill"):
         getattr(L, name).restype = I
@@ -307,6 +313,28 @@ def qsa_sparse_attn_decode(q, k_pages, v_pages, page_table, tok, n_tok, out, wor
                       sm_scale, lse)
     _check(lib().qsa_sparse_attn_decode(*args, _ptr(workspace), ws_bytes, _ptr(dev_status),
                                         _stream(stream)))
+    return out
+
+
+def qsa_sparse_attn_decode_sel_workspace_size(T, Hq, Hkv, D, W, kv_dtype=QSA_BF16) -> int:
+    if isinstance(kv_dtype, torch.dtype):
+        kv_dtype = _dt(torch.empty(0, dtype=kv_dtype))
+    return int(lib().qsa_sparse_attn_decode_sel_workspace_size(T, Hq, Hkv, D, W, kv_dtype))
+
+
+def qsa_sparse_attn_decode_sel(q, k_pages, v_pages, page_table, sel, n_sel, q_pos, W, out, workspace=None,
+                               capture_pos=None, k_scale=1.0, v_scale=1.0, q_req=None, sm_scale=0.0, lse=None,
+                               dev_status=None, stream=None):
+    """Stages 3 and 4 in one call: the decode attention over the tokens the
+    selection sel [T, K] / n_sel [T] expands to (plus 4*c(p0) .. p), W wide."""
+    T, Hq, D = q.shape
+    num_pages, _, Hkv, _ = k_pages.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().qsa_sparse_attn_decode_sel(
+        _ptr(q), _dt(q), _ptr(k_pages), _ptr(v_pages), _dt(k_pages), float(k_scale), float(v_scale), num_pages,
+        _ptr(page_table), page_table.shape[0], page_table.shape[1], _ptr(q_req), _ptr(sel), _ptr(n_sel),
+        sel.shape[1], _ptr(q_pos), _ptr(capture_pos), int(W), T, Hq, Hkv, D, float(sm_scale), _ptr(out), _dt(out),
+        _ptr(lse), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream)))
     return out
 
 

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(L):
     for n in declared_symbols():
         assert hasattr(L, n), n
     assert set(qsa.ENTRY_POINTS) <= set(declared_symbols())
-    assert L.qsa_abi_version() == 10
+    assert L.qsa_abi_version() == 11
 
 
 def test_library_has_no_torch_or_python_dependency():
@@ -145,6 +145,32 @@ def test_decode_workspace_is_checked(L):
     ok = ctypes.c_void_p(0x10000)
     st = _attn(L, "decode", T=1, W=8196, ptr=ok, ws=ok, ws_bytes=need - 16)
     assert st == 3 and str(need) in _err(L)
+
+
+def test_decode_sel_validation(L):
+    """The fused stage 3 + 4 call: W below 4K + 4 and a missing or short
+    workspace are refused on the host, before any launch."""
+    P, I, F, U = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    f = L.qsa_sparse_attn_decode_sel
+    f.argtypes = [P, I, P, P, I, F, F, I, P, I, I, P, P, P, I, P, P, I, I, I, I, I, F, P, I, P, P, U, P, P]
+    L.qsa_sparse_attn_decode_sel_workspace_size.restype = U
+    L.qsa_sparse_attn_decode_sel_workspace_size.argtypes = [I, I, I, I, I, I]
+    ok = ctypes.c_void_p(0x10000)
+
+    def call(K=512, W=2052, T=8, ws=ok, ws_bytes=1 << 30):
+        # (q, q_dt, k, v, kv_dt, ks, vs, pages, pt, pt_rows, pt_stride, q_req, sel, n_sel, K, q_pos, cap,
+        #  W, T, Hq, Hkv, D, sm_scale, out, out_dt, lse, ws, ws_bytes, status, stream)
+        return f(ok, 1, ok, ok, 2, 1.0, 1.0, 4096, ok, 8, 4096, NULL, ok, ok, K, ok, NULL, W, T, 16, 2, 256, 0.0,
+                 ok, 1, NULL, ws, ws_bytes, NULL, NULL)
+    assert call(W=2051) == 1 and "W must be" in _err(L)
+    assert call(K=0) == 1
+    need = L.qsa_sparse_attn_decode_sel_workspace_size(8, 16, 2, 256, 2052, 2)
+    assert need == L.qsa_sparse_attn_decode_workspace_size(8, 16, 2, 256, 2052, 2)   # the gather plan
+    assert call(ws_bytes=need - 16) == 3 and str(need) in _err(L)
+    assert call(ws=NULL) == 3
+    # many rows: the token lists go through the workspace too
+    big = L.qsa_sparse_attn_decode_sel_workspace_size(200, 16, 2, 256, 2052, 2)
+    assert big >= 200 * 2052 * 4
 
 
 def test_binding_refuses_to_run_without_the_library(monkeypatch, tmp_path):

@@ -448,10 +448,14 @@ def test_mtp_draft_loop(oracle, ctx, B, kv):
     w = wl.make("mtp_capture", B=B, ctx=ctx, Hq=16, Hkv=2, D=256, H_I=4, D_I=128, K=512, kv_dtype=kv,
                 q_dtype="bf16", dist="peaked", pages="perm", device="cuda", q_pos=pos,
                 q_req=torch.arange(B, dtype=torch.int32))
-    loop = QSADraftLoop(w, drafts=2)
+    loop = QSADraftLoop(w, drafts=2, fused=False)     # the token lists are written: check them
     loop.run()
+    fused = QSADraftLoop(w, drafts=2)                 # one call per draft step, same outputs bit for bit
+    fused.run()
     torch.cuda.synchronize()
-    assert int(loop.status.item()) == 0
+    assert int(loop.status.item()) == 0 and int(fused.status.item()) == 0
+    for i in range(loop.drafts):
+        assert torch.equal(fused.out[i], loop.out[i]) and torch.equal(fused.lse[i], loop.lse[i])
     n = {k: host(getattr(w, k)) for k in ("page_table", "q_req", "q_pos")}
     sel, n_sel = host(loop.capture.sel), host(loop.capture.n_sel)
     for i in range(loop.drafts):
