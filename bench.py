@@ -286,8 +286,9 @@ def time_e2e(sets, steps, warmup, stream, graph=True):
     cache and the indexer keys are resident device state.
     graph=True: the K timed steps are one captured CUDA graph (the calls'
     host work happens once, at capture).  graph=False: every step issues its
-    copies and library calls from the host inside the timed region (ctypes,
-    argument checks and launches included)."""
+    copies and library calls from the host inside the timed region, the
+    calls bound once by QSAStep.bind (their C argument checks and launches
+    included, the Python argument conversion not)."""
     hosts = []
     for st in sets:
         if not hasattr(st, "_e2e_buffers"):
@@ -298,6 +299,9 @@ def time_e2e(sets, steps, warmup, stream, graph=True):
     d2h = hosts[0][2].numel() * hosts[0][2].element_size()
     cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
     n = len(sets)
+    # eager: each step's library calls are bound once (QSAStep.bind) and
+    # issued from the host every step; the graph captures run() itself
+    bound = [st.bind(stream) for st in sets] if not graph else None
 
     def steps_on(main, count):
         ev_h = [torch.cuda.Event() for _ in range(count)]
@@ -316,7 +320,10 @@ def time_e2e(sets, steps, warmup, stream, graph=True):
             main.wait_event(ev_h[i])
             if i >= n:
                 main.wait_event(ev_d[i - n])      # this set's previous output has been copied out
-            st.run(main)
+            if bound is not None and main is stream:
+                bound[i % n]()
+            else:
+                st.run(main)
             ev_k[i].record(main)
             with torch.cuda.stream(cout):
                 cout.wait_event(ev_k[i])
@@ -443,7 +450,9 @@ def gpu_arm(args):
                       "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                       "ms_per_step": round(e2e_eager_ms / args.steps, 5),
                       "how": "as e2e, but every step's copies and qsa_* calls are issued from the "
-                             "host inside the timed region (no graph)"},
+                             "host inside the timed region (no graph); the calls bound once by "
+                             "QSAStep.bind, so the C argument checks and launches are timed and the "
+                             "Python argument conversion is not"},
         "gpu_launches": (KERNELS_PER_STEP + (1 if sets[0].ws_bytes else 0)) * args.steps,
         "clocks": clk.summary(),
     }

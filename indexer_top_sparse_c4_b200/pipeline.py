@@ -116,6 +116,15 @@ class QSAStep:
         self.attention(stream, sm_scale)
         return self.out
 
+    def bind(self, stream=None, sm_scale=0.0):
+        """run()'s library calls with their arguments converted once: a
+        callable that only crosses into C (for loops where the host issues
+        every step).  It names this step's tensors as they are now: bind
+        again after replacing one; refilling them in place is fine."""
+        if stream is None:
+            stream = torch.cuda.current_stream()
+        return qsa.bind(self.run, stream, sm_scale)
+
 
 class QSADecodeGraphs:
     """The two decode graph families of the sequence-length threshold

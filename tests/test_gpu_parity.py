@@ -82,6 +82,27 @@ def _check_step(oracle, w, step, rows=None, check_scores=True):
     return dict(max_abs=mx, mean_abs=mean, rel_l2=rel)
 
 
+def test_bound_step_equals_run():
+    """QSAStep.bind: the step's calls with their arguments converted once
+    give run()'s outputs bit for bit, refilled inputs included."""
+    w = wl.b1_16k(device="cuda", B=2, kv_dtype="fp8")
+    st = QSAStep(w)
+    step = st.bind()
+    st.run()
+    ref = (st.out.clone(), st.lse.clone(), st.tok.clone())
+    st.out.zero_()
+    st.tok.zero_()
+    step()
+    torch.cuda.synchronize()
+    assert torch.equal(st.out, ref[0]) and torch.equal(st.lse, ref[1]) and torch.equal(st.tok, ref[2])
+    w.q.copy_(torch.flip(w.q, dims=[0]))          # new inputs, same tensors
+    step()
+    out_b = st.out.clone()
+    st.run()
+    torch.cuda.synchronize()
+    assert torch.equal(out_b, st.out) and int(st.status.item()) == 0
+
+
 def test_tiny_decode(oracle):
     w = wl.tiny(device="cuda")
     _check_step(oracle, w, QSAStep(w))
