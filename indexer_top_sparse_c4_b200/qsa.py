@@ -77,7 +77,8 @@ def bind(fn, *args, **kwargs):
     crosses into C, for host-bound loops.  The tensors and the stream the
     calls name are fixed at binding: they must stay allocated and in place
     (bind again after replacing one), and ``stream=None`` means the stream
-    current now."""
+    current now.  Bind from one thread at a time: while ``fn`` runs, lib()
+    hands out the recorder."""
     global _binding
     rec = _Recorder(lib())
     _binding = rec

@@ -173,6 +173,34 @@ def test_decode_sel_validation(L):
     assert big >= 200 * 2052 * 4
 
 
+def test_bind_records_launches_and_checks_them_when_called(L):
+    """qsa.bind: the wrapped wrapper runs once with the library's launching
+    calls recorded, not made; the bound call makes them, and a call the
+    library refuses raises then, not at binding.  Size queries are answered
+    at binding and not recorded."""
+    import torch
+    from indexer_top_sparse_c4_b200 import qsa
+
+    class Stream:
+        cuda_stream = 0
+
+    scores = torch.zeros((1, 8))
+    q_pos = torch.zeros((1,), dtype=torch.int32)
+    sel = torch.zeros((1, 1), dtype=torch.int32)
+    n_sel = torch.zeros((1,), dtype=torch.int32)
+    call = qsa.bind(qsa.qsa_topk_groups_gvr, scores, q_pos, 0, sel, n_sel, stream=Stream())   # K = 0
+    with pytest.raises(qsa.QSAError, match="K must be"):
+        call()
+    empty = torch.zeros((0, 4), dtype=torch.int32)
+    qsa.bind(qsa.qsa_dense_select, torch.zeros((0,), dtype=torch.int32), 100, empty,
+             torch.zeros((0,), dtype=torch.int32), stream=Stream())()          # T = 0: nothing to launch
+    sizes = []
+    nothing = qsa.bind(lambda: sizes.append(qsa.qsa_sparse_attn_decode_workspace_size(8, 16, 2, 256, 2052, 2)))
+    assert sizes == [L.qsa_sparse_attn_decode_workspace_size(8, 16, 2, 256, 2052, 2)] and sizes[0] > 0
+    nothing()
+    assert qsa.lib() is L                                # binding leaves the library in place
+
+
 def test_binding_refuses_to_run_without_the_library(monkeypatch, tmp_path):
     from indexer_top_sparse_c4_b200 import qsa
     monkeypatch.setattr(qsa, "LIB_PATH", str(tmp_path / "libqsa.so"))
