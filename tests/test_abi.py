@@ -201,6 +201,30 @@ def test_bind_records_launches_and_checks_them_when_called(L):
     assert qsa.lib() is L                                # binding leaves the library in place
 
 
+@pytest.mark.parametrize("T, Hq, Hkv, D, W, kv, parts", [
+    (8, 16, 2, 256, 2052, 2, 9),      # B8, K=512: 16 rows, one CTA per SM -> 9 chunks per row
+    (8, 16, 2, 256, 8196, 2, 9),      # K=2,048: the same 9 chunks, longer
+    (8, 16, 2, 256, 16388, 2, 17),    # K=4,096: the row-index table (1,024 slots) forces 17 chunks
+    (40, 16, 2, 256, 2052, 2, 3),     # 80 rows: one per SM would do, the table asks for 3
+    (40, 16, 2, 256, 516, 2, 1),      # 80 rows of 516 slots: one chunk each, no partials
+    (80, 16, 2, 256, 2052, 2, 1),     # 160 rows: the streaming kernel, no partials
+    (1, 4, 1, 64, 132, 0, 3),         # FP32 / D=64: the general kernel, split in 64-slot pieces
+])
+def test_decode_plan_through_the_workspace_query(L, T, Hq, Hkv, D, W, kv, parts):
+    """The decode attention's plan, seen through its workspace: T * Hq
+    partials of (D + 2) floats per chunk (or split) of a row, none when a
+    row is not split."""
+    need = L.qsa_sparse_attn_decode_workspace_size(T, Hq, Hkv, D, W, kv)
+    assert need == (0 if parts == 1 else T * Hq * parts * (D + 2) * 4)
+    sel = L.qsa_sparse_attn_decode_sel_workspace_size(T, Hq, Hkv, D, W, kv)
+    gather = kv != 0 and T * Hkv < 148
+    if gather:   # the gather kernel lists its tokens itself
+        assert sel == need
+    else:        # the token lists go through the workspace
+        a16 = lambda n: (n + 15) // 16 * 16
+        assert sel == a16(need) + a16(T * W * 4) + a16(T * 4)
+
+
 def test_binding_refuses_to_run_without_the_library(monkeypatch, tmp_path):
     from indexer_top_sparse_c4_b200 import qsa
     monkeypatch.setattr(qsa, "LIB_PATH", str(tmp_path / "libqsa.so"))
