@@ -172,10 +172,12 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
     nt = 0;
   }
   const int32_t* pt = a.page_table + (size_t)r * a.pt_stride;
+  // the chunk slots [lo, hi) of the row-index table: token id -> page -> row
+  auto resolve = [&](int lo, int hi) {
 #pragma unroll
   for (int k = 0; k < IPT; ++k) {
     const int i = tid + k * NTHR;
-    if (i < C) {
+    if (i >= lo && i < hi) {
       const int j = cbeg + i < nt ? jv[k] : -1;
       int ri = -1;
       if (j < -1 || (j >= 0 && j / kPageTokens >= a.pt_stride)) {
@@ -191,6 +193,11 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
       tbl[i] = ri;
     }
   }
+  };
+  // first the slots of every slot's first NS - 1 tiles (those are issued
+  // before the loop); the rest while their copies are in flight
+  const int c_first = C < 16 * SL * (NS - 1) ? C : 16 * SL * (NS - 1);
+  resolve(0, c_first);
 
   // ---- Q^T B fragments of heads h0 + 8u + g (zero past G), head dim permuted
   // like K: k-steps j * KS .. j * KS + KS - 1 take dims CH (4j + tq) + 0..CH-1,
@@ -218,7 +225,7 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
       }
     }
   }
-  __syncthreads();  // the row-index table is complete
+  __syncthreads();  // the first tiles' rows are in the table
 
   const int clen = nt - cbeg < C ? nt - cbeg : C;             // slots of this chunk in the list
   const int ntiles = clen > 0 ? (clen + 15) / 16 : 0;          // tiles of the chunk
@@ -260,6 +267,10 @@ __global__ void __launch_bounds__(ga_slots(FP8, NT) * NT * 32, 1)
   };
 #pragma unroll
   for (int i = 0; i < NS - 1; ++i) issue(i);
+  if (c_first < C) {
+    resolve(c_first, C);
+    __syncthreads();  // the rest of the table is complete
+  }
 
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f, o[MT][4];
 #pragma unroll
