@@ -607,6 +607,12 @@ def prefill_summary(device, stream, seed, reps):
             g.replay()
             times[name] = replay_ms(g) / reps
             del g
+    # the Top-K alone on the chunk's scores: radix passes against the
+    # guess-verify-refine mode (same selection; the step uses the radix kernel)
+    from indexer_top_sparse_c4_b200 import qsa
+    sel2, n2 = torch.empty_like(st.sel), torch.empty_like(st.n_sel)
+    topk_radix_us = graph_us(lambda i: qsa.qsa_topk_groups(st.scores, st.sel_pos, w.K, sel2, n2), reps, stream)
+    topk_gvr_us = graph_us(lambda i: qsa.qsa_topk_groups_gvr(st.scores, st.sel_pos, w.K, sel2, n2), reps, stream)
     sum_c = int((w.q_pos // 4).sum().item())
     sum_tok = int(st.n_tok.sum().item())
     idx_flop = 2.0 * w.H_I * w.D_I * sum_c
@@ -626,6 +632,7 @@ def prefill_summary(device, stream, seed, reps):
         "query_tokens_per_s": round(w.T / (times["step"] / 1e3), 1),
         "ms_per_step": round(times["step"], 4),
         "stages_ms": {names[k]: round(times[k], 4) for k in STAGES},
+        "topk_alone_ms": {"radix": round(topk_radix_us / 1e3, 4), "gvr": round(topk_gvr_us / 1e3, 4)},
         "index_scores": {"bound": "tensor", "flop_per_launch": idx_flop,
                          "achieved": round(idx_tf, 1), "peak": peak, "peak_kind": kind,
                          "unit": "TFLOP/s", "frac": round(idx_tf / peak, 4)},

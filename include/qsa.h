@@ -200,14 +200,14 @@ QSA_API qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint
  * of the row's own scores where the K-th largest lies, verifies the guess by
  * exact counts, and refines with an exact select among the candidates the
  * guess leaves; a row whose guess fails takes a radix select over the whole
- * row.  Few long rows (under 148 rows of more than 8,192 candidates: decode)
- * run on one thread-block cluster per row: the guess is a window of key bins
- * around the sample's rank of the K-th key, the counts above and in it are
- * exact over the cluster.  Many rows run one CTA per row: the guess is a
- * threshold, re-guessed from the sample up to twice when its count is too
- * small or too large.  path (optional, [T] int32) receives per row: 0 dense
- * (c <= K), 1 the first guess verified, 2 a later guess verified, 3 the
- * whole-row select.
+ * row.  The guess is a window of 12-bit key bins around the sample's rank of
+ * the K-th key; the counts of the keys above and in it are exact, and the
+ * select runs over the window's keys alone.  Rows run as qsa_topk_groups
+ * runs them: one CTA per row for many rows (148 or more) of up to 32,768
+ * candidates and for rows of up to 8,192, one thread-block cluster per row
+ * otherwise (decode).  score_stride at most 262,144.  path (optional, [T]
+ * int32) receives per row: 0 dense (c <= K), 1 the guess verified, 3 the
+ * radix select over the whole row.
  * For K outside {512, 1024, 2048} the call runs qsa_topk_groups instead (a
  * message on stderr the first time) and leaves path unwritten. */
 QSA_API qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K,

@@ -291,7 +291,7 @@ qsa_status_t qsa_topk_groups(const float* scores, int score_stride, uint32_t* pr
   REQUIRE(K >= 1, "K must be >= 1 (got %d)", K);
   REQUIRE(score_stride >= 1, "score_stride must be >= 1");
   SUPPORT(qsa::topk_cluster_size(score_stride) > 0, "score_stride %d exceeds the %d groups a row may hold",
-          score_stride, 8 * 49152);
+          score_stride, 8 * 512 * 64);
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
   REQUIRE(aligned16(prefix_hist), "prefix_hist must be 16-byte aligned");
@@ -318,17 +318,17 @@ qsa_status_t qsa_topk_groups_gvr(const float* scores, int score_stride, const in
     }
     return qsa_topk_groups(scores, score_stride, nullptr, q_pos, T, K, sel, n_sel, nullptr, 0, dev_status, stream);
   }
+  SUPPORT(qsa::topk_cluster_size(score_stride) > 0, "score_stride %d exceeds the %d groups a row may hold",
+          score_stride, 8 * 512 * 64);
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel, "null pointer argument");
-  if (T < 148 && qsa::topk_cluster_size(score_stride) > 1) {
-    // few long rows (decode): the cluster Top-K with the self-sampled guess
-    qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
-    a.gvr = 1;
-    a.path = path;
-    return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups_gvr launch");
-  }
-  return cuda_status(qsa::launch_topk_gvr(scores, score_stride, q_pos, T, K, sel, n_sel, path, (cudaStream_t)stream),
-                     "qsa_topk_groups_gvr launch");
+  // the Top-K kernels of stage 2 with the self-sampled guess in front of
+  // their radix passes: one CTA per row (many rows, or short ones), one
+  // cluster per row (few long rows)
+  qsa::TopkArgs a{scores, score_stride, q_pos, T, K, sel, n_sel, dev_status};
+  a.gvr = 1;
+  a.path = path;
+  return cuda_status(qsa::launch_topk_groups(a, (cudaStream_t)stream), "qsa_topk_groups_gvr launch");
 }
 
 qsa_status_t qsa_expand_select(const int32_t* sel, const int32_t* n_sel, int K, const int32_t* q_pos,
@@ -371,7 +371,7 @@ qsa_status_t qsa_topk_expand(const float* scores, int score_stride, uint32_t* pr
   REQUIRE(W >= 4 * K + 4, "W must be >= 4*K + 4 = %d (got %d)", 4 * K + 4, W);
   REQUIRE(score_stride >= 1, "score_stride must be >= 1");
   SUPPORT(qsa::topk_cluster_size(score_stride) > 0, "score_stride %d exceeds the %d groups a row may hold",
-          score_stride, 8 * 49152);
+          score_stride, 8 * 512 * 64);
   if (T == 0) return QSA_OK;
   REQUIRE(scores && q_pos && sel && n_sel && tok && n_tok, "null pointer argument");
   REQUIRE(aligned16(prefix_hist), "prefix_hist must be 16-byte aligned");

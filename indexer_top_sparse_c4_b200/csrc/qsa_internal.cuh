@@ -224,9 +224,9 @@ struct TopkArgs {
   // optional [T][kPrefixBins] prefix histogram from the scan: read in place of
   // the first cluster passes where a row's total matches, then zeroed
   uint32_t* hist = nullptr;
-  // guess-verify-refine with self-sampling (cluster kernel, no histogram): the
-  // guess is a window of key bins read off a strided sample of the row;
-  // path (optional) gets 0 dense, 1 the guess verified, 3 the cluster passes
+  // guess-verify-refine with self-sampling (no histogram; row and cluster
+  // kernels): the guess is a window of key bins read off a strided sample of
+  // the row; path (optional) gets 0 dense, 1 the guess verified, 3 the radix passes
   int gvr = 0;
   int32_t* path = nullptr;
 };
@@ -305,10 +305,8 @@ cudaError_t launch_compress_keys(const CompressArgs& c, qsa_dtype_t k_dt, cudaSt
 // Self-test of the bounded mbarrier wait (selftest.cu).
 cudaError_t launch_selftest_wait(uint32_t limit_us, uint32_t* status, uint32_t* report, cudaStream_t s);
 
-// Guess-verify-refine Top-K with self-sampling (topk_gvr.cu).
+// Budgets the guess-verify-refine Top-K serves (topk_groups.cu, TopkArgs::gvr).
 bool topk_gvr_budget(int K);
-cudaError_t launch_topk_gvr(const float* scores, int score_stride, const int32_t* q_pos, int T, int K, int32_t* sel,
-                            int32_t* n_sel, int32_t* path, cudaStream_t s);
 
 // Sequence-sharded decode (dcp.cu).
 cudaError_t launch_dcp_positions(const int32_t* q_pos, int T, int g_lo, int g_hi, int32_t* q_pos_local,

@@ -15,7 +15,12 @@
 // Two kernels:
 //  * topk_row_kernel (many rows, e.g. a prefill chunk): one CTA per row, keys
 //    in registers, four block-local passes.  Many CTAs per SM keep the code
-//    hot in the instruction caches.
+//    hot in the instruction caches.  In its guess-verify-refine mode (no
+//    hint) the passes over the whole row give way to a self-sampled guess:
+//    a histogram of the top 12 key bits of every (KPT/4)-th key gives a
+//    window of bins around the n-th key's sample rank, one pass counts the
+//    keys above and in it, and when the counts confirm it the digit passes
+//    run over the window's keys alone.
 //  * topk_cluster_kernel (few long rows, decode): one thread-block cluster of
 //    CL CTAs per row.  Each code path runs once per launch, so the kernel is
 //    written for a small instruction footprint: keys live in shared memory
@@ -341,11 +346,119 @@ __device__ __forceinline__ int count_vs(const Keys& keys, uint32_t tau) {
   return gt | (eq << 16);
 }
 
-// ---- many rows: one CTA per row, keys in registers --------------------------------
+// Guess-verify-refine for one CTA's row, keys in registers: the key tau of the
+// n-th largest candidate and how many keys equal to tau are kept, without the
+// four radix passes over the whole row.  Thread i samples its keys 0, KPT/4,
+// KPT/2, 3KPT/4, i.e. every (KPT/4)-th id of the row; a histogram of their
+// top 12 key bits gives the window of bins between the sample ranks
+// n ns / c -+ (3 sigma + 1).  One pass counts the keys above the window and
+// in it; when those exact counts put the n-th key inside the window (and the
+// window holds at most kListCapG keys), the window's keys are listed with their
+// ids and four digit passes over them alone find tau (the window bin, then
+// bits 12..19, 4..11 and 0..3).  Returns false, with nothing written, when the
+// guess fails; the caller then runs the radix passes.  (Block-uniform.)
 template <int KPT>
+__device__ __forceinline__ bool row_guess(TopkSmemG& sm, const RegKeys<KPT>& keys, int first, int c, int n,
+                                          uint32_t& tau, int& need) {
+  static_assert(KPT % 4 == 0 && kThreads * 8 == kPrefixBins, "4 samples per thread, 8 bins per thread");
+  constexpr int SS = KPT / 4;  // sample stride
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* const sh = &sm.hw[0][0];  // the 4,096-bin sample histogram (flat)
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sh[8 * tid + j] = 0u;
+  if (tid == 0) {
+    sm.pbin = kPrefixBins - 1;
+    sm.pbin_lo = 0;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < 4; ++m)
+    if (first + m * SS < c) atomicAdd(&sh[keys.get(m * SS) >> kPrefixShift], 1u);
+  __syncthreads();
+  const int ns = (c + SS - 1) / SS;  // sampled ids: the multiples of SS below c
+  int hs = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) hs += (int)sh[kPrefixBins - 1 - 8 * tid - j];
+  int htotal;
+  const int hbefore = block_exclusive_scan(hs, sm.wa, htotal);
+  const float e = (float)n * (float)ns / (float)c, sd = sqrtf(e);
+  const int r_hi = max(1, (int)floorf(e - 3.f * sd - 1.f));
+  const int r_lo = min(ns, (int)ceilf(e + 3.f * sd + 1.f));
+  int ab = hbefore;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // (the counts are read again: fewer registers live across the scan)
+    const int b = kPrefixBins - 1 - 8 * tid - j;
+    const int h = (int)sh[b];
+    if (ab < r_hi && ab + h >= r_hi) sm.pbin = b;
+    if (ab < r_lo && ab + h >= r_lo) sm.pbin_lo = b;
+    ab += h;
+  }
+  __syncthreads();
+  const uint32_t pb = (uint32_t)sm.pbin, pb_lo = (uint32_t)sm.pbin_lo;
+  if (pb - pb_lo >= (uint32_t)kBins) return false;  // the window does not fit one 256-bin pass
+
+  // ---- verify: exact counts above the window and in it
+  int mine = 0, above = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const uint32_t b = keys.get(j) >> kPrefixShift;
+    const bool valid = first + j < c;
+    above += valid && b > pb;
+    mine += valid && b <= pb && b >= pb_lo;
+  }
+  int tot;  // candidates (low 16 bits; c <= 32,768) and keys above the window (high)
+  int pos = block_exclusive_scan(mine | (above << 16), sm.wa, tot) & 0xffff;
+  const int in_win = tot & 0xffff, above_all = tot >> 16;
+  if (!(above_all < n && above_all + in_win >= n && in_win <= kListCapG)) return false;
+
+  // ---- refine: the window's keys with their ids, in id order
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const uint32_t k = keys.get(j), b = k >> kPrefixShift;
+    if (first + j < c && b <= pb && b >= pb_lo) sm.cand[pos++] = make_uint2(k, (uint32_t)(first + j));
+  }
+  __syncthreads();
+  uint32_t pre = 0;
+  int nd = n - above_all;  // the nd-th largest in the window is the n-th of the row
+#pragma unroll 1
+  for (int pass = 0; pass < 4; ++pass) {
+    // pass 0: the window bin (offset from pb_lo); then bits 12..19, 4..11, 0..3
+    const int shift = pass == 0 ? kPrefixShift : (pass == 1 ? 12 : (pass == 2 ? 4 : 0));
+    const int fixed = pass == 1 ? kPrefixShift : (pass == 2 ? 12 : 4);  // bits above `shift` already known
+    const uint32_t dmask = pass == 3 ? 0xFu : 0xFFu;
+#pragma unroll
+    for (int b = lane; b < kBins; b += 32) sm.hw[warp][b] = 0u;
+    __syncwarp();
+    for (int i = tid; i < in_win; i += kThreads) {
+      const uint32_t k = sm.cand[i].x;
+      if (pass == 0) atomicAdd(&sm.hw[warp][(k >> kPrefixShift) - pb_lo], 1u);
+      else if ((k >> fixed) == (pre >> fixed)) atomicAdd(&sm.hw[warp][(k >> shift) & dmask], 1u);
+    }
+    __syncthreads();
+    if (tid < kBins) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
+      find_bin((int)v, nd, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+    }
+    __syncthreads();
+    const uint32_t d = (uint32_t)sm.bin[pass];
+    pre |= pass == 0 ? (pb_lo + d) << kPrefixShift : d << shift;
+    nd -= sm.above[pass];
+  }
+  tau = pre;
+  need = nd;
+  return true;
+}
+
+// ---- many rows: one CTA per row, keys in registers --------------------------------
+// GVR: first the self-sampled guess of row_guess (guess-verify-refine), the
+// radix passes only when it fails.
+template <int KPT, bool GVR>
 __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int vec, int tvec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(smem_raw);
+  using SMT = TopkSmemT<GVR ? kListCapG : kCandCap>;
+  SMT& sm = *reinterpret_cast<SMT*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int t = blockIdx.y;
   pdl_wait();
@@ -361,31 +474,35 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
   // (dependents launch when this grid completes: launched earlier, their CTAs
   // compete for the SMs this kernel still needs)
 
-  // ---- radix select: four passes of 8 bits from the top
   uint32_t prefix = 0;
   int need = r.n;  // how many keys matching `prefix` are still to be taken
+  bool guessed = false;
+  if constexpr (GVR) guessed = row_guess<KPT>(sm, keys, first, r.c, r.n, prefix, need);
+  // ---- radix select: four passes of 8 bits from the top
+  if (!guessed) {
 #pragma unroll
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
 #pragma unroll
-    for (int b = threadIdx.x & 31; b < kBins; b += 32) sm.hw[warp][b] = 0u;
-    __syncwarp();
+      for (int b = threadIdx.x & 31; b < kBins; b += 32) sm.hw[warp][b] = 0u;
+      __syncwarp();
 #pragma unroll
-    for (int j = 0; j < KPT; ++j) {
-      const uint32_t k = keys.get(j);
-      const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
-      if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
+      for (int j = 0; j < KPT; ++j) {
+        const uint32_t k = keys.get(j);
+        const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
+        if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
+      }
+      __syncthreads();
+      if (tid < kBins) {
+        uint32_t v = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
+        find_bin((int)v, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+      }
+      __syncthreads();
+      prefix |= (uint32_t)sm.bin[pass] << shift;
+      need -= sm.above[pass];
     }
-    __syncthreads();
-    if (tid < kBins) {
-      uint32_t v = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
-      find_bin((int)v, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
-    }
-    __syncthreads();
-    prefix |= (uint32_t)sm.bin[pass] << shift;
-    need -= sm.above[pass];
   }
   const uint32_t tau = prefix;
 
@@ -396,6 +513,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
   emit_kept<KPT, false>(sm, keys, 0, 0, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff,
                         both >> 16, need, 0, r, tvec);
   write_tail(a, r, t);
+  if (GVR && tid == 0 && a.path) a.path[t] = guessed ? 1 : 3;
 }
 
 // ---- few long rows: one cluster per row, keys in shared memory ------------------
@@ -909,8 +1027,8 @@ cudaError_t launch_cfg(const TopkArgs& a, cudaStream_t s) {
   const int vec = (a.score_stride % 4 == 0) && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
   const int tvec = a.tok && a.W % 4 == 0 && (reinterpret_cast<uintptr_t>(a.tok) & 15u) == 0;
   if constexpr (CL == 1) {
-    const size_t smem = sizeof(TopkSmem);
-    auto kern = topk_row_kernel<KPT>;
+    const size_t smem = a.gvr ? sizeof(TopkSmemG) : sizeof(TopkSmem);
+    auto kern = a.gvr ? topk_row_kernel<KPT, true> : topk_row_kernel<KPT, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_k(kern, dim3(1, a.T), dim3(kThreads), smem, s, 1, a, vec, tvec);
@@ -956,6 +1074,8 @@ TopkPlan plan_for(int T, int score_stride) {
 }  // namespace
 
 int topk_cluster_size(int score_stride) { return plan_for(1, score_stride).cl; }
+
+bool topk_gvr_budget(int K) { return K == 512 || K == 1024 || K == 2048; }
 
 cudaError_t launch_topk_groups(const TopkArgs& a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;

@@ -93,6 +93,12 @@ def test_topk_validation(L):
     assert L.qsa_topk_groups(NULL, 10 ** 7, NULL, NULL, 2, 4, NULL, NULL, NULL, 0, NULL, NULL) == 2
     assert L.qsa_topk_groups(NULL, 16, NULL, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 0
     assert L.qsa_topk_groups_workspace_size(8, 512, 65535) == 0
+    # rows of up to 262,144 candidates (8 CTAs x 512 threads x 64 keys)
+    assert L.qsa_topk_groups(NULL, 262144, NULL, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 0
+    assert L.qsa_topk_groups(NULL, 262145, NULL, NULL, 0, 4, NULL, NULL, NULL, 0, NULL, NULL) == 2
+    assert L.qsa_topk_groups_gvr(NULL, 262144, NULL, 0, 512, NULL, NULL, NULL, NULL, NULL) == 0
+    assert L.qsa_topk_groups_gvr(NULL, 262145, NULL, 0, 512, NULL, NULL, NULL, NULL, NULL) == 2
+    assert L.qsa_topk_groups_gvr(NULL, 16, NULL, 2, 512, NULL, NULL, NULL, NULL, NULL) == 1   # null pointers
 
 
 def test_expand_validation(L):

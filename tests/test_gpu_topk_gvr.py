@@ -145,3 +145,57 @@ def test_gvr_other_budgets_use_the_radix_top_k(q):
     rs, rn = _radix(q, st.scores, w.q_pos, 300)
     assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
     assert host(path).tolist() == [-1]          # untouched: the radix Top-K ran
+
+
+def _rows_scores(T, stride, c, dist, seed):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    s = torch.randn((T, stride), generator=g)
+    if dist == "peaked":     # 5% of the groups 3 sigma up
+        s += 3.0 * (torch.rand((T, stride), generator=g) < 0.05).float()
+    elif dist == "ties":     # 16 levels
+        s = torch.randint(0, 16, (T, stride), generator=g).float()
+    q_pos = torch.full((T,), 4 * c + 2, dtype=torch.int32)
+    return s.cuda(), q_pos.cuda()
+
+
+@pytest.mark.parametrize("stride", [4096, 16384, 32768])     # 8, 32 and 64 keys per thread
+@pytest.mark.parametrize("dist", ["normal", "peaked", "ties"])
+def test_gvr_many_rows_one_cta_each(q, oracle, stride, dist):
+    """Many rows (one CTA each, keys in registers): the self-sampled window
+    selects on ordinary rows, bit for bit the radix Top-K and the oracle, at
+    the three budgets; rows of the prefill chunk's length among them."""
+    T, c = 160, stride - 1
+    scores, q_pos = _rows_scores(T, stride, c, dist, seed=stride + len(dist))
+    ref_s = host(scores)
+    for K in (512, 1024, 2048):
+        if K >= c:
+            continue
+        sel, n_sel, path = _gvr(q, scores, q_pos, K)
+        rs, rn = _radix(q, scores, q_pos, K)
+        assert torch.equal(sel, rs) and torch.equal(n_sel, rn), K
+        ref, nref = oracle.topk_groups(ref_s, host(q_pos), K)
+        assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref), K
+        p = host(path)
+        if dist == "ties" or 4 * K > c:   # crowded levels; a K-th key near 0 (its window spans the sign)
+            assert set(p.tolist()) <= {1, 3}, K
+        else:
+            assert np.all(p == 1), (K, np.bincount(p))
+
+
+@pytest.mark.parametrize("K", [512, 2048])
+def test_gvr_many_rows_guess_missed_by_the_sample_is_caught(q, oracle, K):
+    """Rows of 16,383 candidates (32 keys per thread, every 8th id sampled)
+    whose largest scores sit only at ids 3 mod 8: the window lies below
+    them, the exact count above it exceeds the budget, and every row takes
+    the radix passes -- with the exact result."""
+    T, stride = 160, 16384
+    c = stride - 1
+    scores, q_pos = _rows_scores(T, stride, c, "normal", seed=K)
+    hidden = torch.arange(3, c, 8)[: K + 100]
+    scores[:, hidden.cuda()] = 50.0
+    sel, n_sel, path = _gvr(q, scores, q_pos, K)
+    assert np.all(host(path) == 3)
+    rs, rn = _radix(q, scores, q_pos, K)
+    assert torch.equal(sel, rs) and torch.equal(n_sel, rn)
+    ref, nref = oracle.topk_groups(host(scores), host(q_pos), K)
+    assert np.array_equal(host(sel), ref) and np.array_equal(host(n_sel), nref)
