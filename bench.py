@@ -815,6 +815,71 @@ def reference_arm(args):
     }
 
 
+def oracle_configs_arm(args):
+    """`--impl reference --oracle-configs`: the oracle as it stands on the host
+    cores, over every config: tiny, B1 16K, B8 262K at the three budgets, the
+    prefill chunk (64 of its query rows, or all of them with
+    --oracle-full-prefill) and the sweep's covering cases.  Each is timed with
+    the oracle's OpenMP loop over query rows on every core it can use, and on
+    one core, each for about --cpu-seconds / 4.  Host work only (the inputs
+    are drawn on the host); one JSON line, a reported baseline."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle as orc
+    from indexer_top_sparse_c4_b200 import workloads as wl
+    orc.build()
+    host_cores = os.cpu_count() or 1
+    secs = max(args.cpu_seconds / 4, 0.5)
+    per_row = ("q", "q_idx", "w_idx", "q_pos", "q_req", "capture_pos")
+
+    def rows_of(n, idx):
+        m = dict(n)
+        for k in per_row:
+            if m.get(k) is not None:
+                m[k] = np.ascontiguousarray(m[k][idx])
+        return m
+
+    def time_config(w, n, K, sample, name=None):
+        T = int(n["q_pos"].shape[0])
+        out = {"workload": name or w.name, "K": K, "rows": T, "threads": min(orc.threads_for(T), host_cores),
+               "sample": sample}
+        for label, threads in (("all_cores", host_cores), ("one_core", 1)):
+            orc.set_max_threads(threads)
+            steps, el = _time_oracle(orc, n, K, w.k_scale, w.v_scale, secs)
+            out[label] = {"tokens_per_s": round(T * steps / el, 3), "steps": steps, "seconds": round(el, 2)}
+        orc.set_max_threads(host_cores)
+        return out
+
+    res = []
+    for make in (lambda: wl.tiny(seed=args.seed), lambda: wl.b1_16k(seed=args.seed)):
+        w = make()
+        res.append(time_config(w, w.numpy(), w.K, "every query row, all four stages"))
+    w = wl.b8_262k(K=2048, seed=args.seed)   # the budgets share the inputs; W fits K = 2,048
+    n = w.numpy()
+    for K in (512, 1024, 2048):
+        res.append(time_config(w, n, K, "every query row (8), all four stages", f"b8_decode_262k_fp8_k{K}"))
+    del w, n
+    w = wl.prefill_chunk(seed=args.seed)
+    n = w.numpy()
+    if args.oracle_full_prefill:
+        res.append(time_config(w, n, w.K, "every query row (8,192), all four stages"))
+    else:
+        idx = np.unique(np.linspace(0, w.T - 1, 64).astype(int))
+        res.append(time_config(w, rows_of(n, idx), w.K,
+                               f"{idx.size} of the {w.T:,} query rows, evenly spaced, all four stages"))
+    del w, n
+    for case in wl.SWEEP_CASES:
+        ctx, B, heads, K, kv, dist = case
+        w = wl.sweep_case(ctx, B, heads, K, kv, dist, seed=ctx + B)
+        res.append(time_config(w, w.numpy(), K, "every query row, all four stages"))
+        del w
+    return {"impl": "reference", "oracle_configs": res, "host_cores": host_cores, "kind": "oracle",
+            "unit": "tokens/s (query rows through all four stages per second)",
+            "note": "inputs drawn on the host (the same recipe and seeds; the GPU arm draws on the GPU)"}
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -837,10 +902,14 @@ def main(argv=None):
                     help="leave out the prefill-chunk summary of the decode line")
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode",
                     help="prefill: time only the 8,192-token prefill chunk (one GPU)")
+    ap.add_argument("--oracle-configs", action="store_true",
+                    help="with --impl reference: time the oracle on every config (host only)")
+    ap.add_argument("--oracle-full-prefill", action="store_true",
+                    help="with --oracle-configs: every query row of the prefill chunk, not 64")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
-        line = reference_arm(args)
+        line = oracle_configs_arm(args) if args.oracle_configs else reference_arm(args)
     elif args.workload == "prefill":
         line = prefill_arm(args)
     else:

@@ -308,6 +308,22 @@ SWEEP_BUDGETS = (512, 1024, 2048)
 SWEEP_KV = ("bf16", "fp8")
 SWEEP_DISTS = ("normal", "peaked", "ties")
 
+# A covering subset of the sweep's cross product (5 x 4 x 4 x 3 x 2 x 3 =
+# 1,440 cases): every value of every axis appears at least once.
+# (context, batch, (Hq, Hkv), budget, KV storage, score distribution)
+SWEEP_CASES = (
+    (4096, 1, (16, 2), 512, "bf16", "ties"),
+    (4096, 8, (3, 1), 2048, "fp8", "normal"),
+    (16384, 2, (12, 1), 1024, "fp8", "peaked"),
+    (16384, 4, (6, 1), 2048, "bf16", "ties"),
+    (65536, 4, (16, 2), 512, "fp8", "normal"),
+    (65536, 1, (3, 1), 1024, "bf16", "peaked"),
+    (131072, 2, (6, 1), 512, "fp8", "ties"),
+    (131072, 8, (12, 1), 2048, "bf16", "normal"),
+    (262144, 1, (16, 2), 2048, "bf16", "ties"),
+    (262144, 2, (12, 1), 1024, "fp8", "peaked"),
+)
+
 
 def sweep_case(ctx, B, heads, K, kv, dist, device="cpu", seed=0) -> Workload:
     Hq, Hkv = heads

@@ -494,18 +494,7 @@ def test_mtp_draft_loop(oracle, ctx, B, kv):
         assert mx <= ATTN_MAX_ABS and mean <= ATTN_MEAN_ABS and rel <= ATTN_REL_L2, (mx, mean, rel)
 
 
-SWEEP = [  # every value of every sweep axis appears at least once
-    (4096, 1, (16, 2), 512, "bf16", "ties"),
-    (4096, 8, (3, 1), 2048, "fp8", "normal"),
-    (16384, 2, (12, 1), 1024, "fp8", "peaked"),
-    (16384, 4, (6, 1), 2048, "bf16", "ties"),
-    (65536, 4, (16, 2), 512, "fp8", "normal"),
-    (65536, 1, (3, 1), 1024, "bf16", "peaked"),
-    (131072, 2, (6, 1), 512, "fp8", "ties"),
-    (131072, 8, (12, 1), 2048, "bf16", "normal"),
-    (262144, 1, (16, 2), 2048, "bf16", "ties"),
-    (262144, 2, (12, 1), 1024, "fp8", "peaked"),
-]
+SWEEP = wl.SWEEP_CASES   # every value of every sweep axis appears at least once
 
 
 @pytest.mark.parametrize("case", SWEEP, ids=lambda c: f"c{c[0]}_b{c[1]}_h{c[2][0]}x{c[2][1]}_k{c[3]}_{c[4]}_{c[5]}")
