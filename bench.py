@@ -818,11 +818,11 @@ def reference_arm(args):
 def oracle_configs_arm(args):
     """`--impl reference --oracle-configs`: the oracle as it stands on the host
     cores, over every config: tiny, B1 16K, B8 262K at the three budgets, the
-    prefill chunk (64 of its query rows, or all of them with
-    --oracle-full-prefill) and the sweep's covering cases.  Each is timed with
-    the oracle's OpenMP loop over query rows on every core it can use, and on
-    one core, each for about --cpu-seconds / 4.  Host work only (the inputs
-    are drawn on the host); one JSON line, a reported baseline."""
+    prefill chunk (64 of its query rows; with --oracle-full-prefill also all
+    of them, once, on every core) and the sweep's covering cases.  Each is
+    timed with the oracle's OpenMP loop over query rows on every core it can
+    use, and on one core, each for about --cpu-seconds / 4.  Host work only
+    (the inputs are drawn on the host); one JSON line, a reported baseline."""
     ws, rank, local = dist_env()
     if rank != 0:
         return None
@@ -841,11 +841,12 @@ def oracle_configs_arm(args):
                 m[k] = np.ascontiguousarray(m[k][idx])
         return m
 
-    def time_config(w, n, K, sample, name=None):
+    def time_config(w, n, K, sample, name=None, modes=(("all_cores", None), ("one_core", 1))):
         T = int(n["q_pos"].shape[0])
         out = {"workload": name or w.name, "K": K, "rows": T, "threads": min(orc.threads_for(T), host_cores),
                "sample": sample}
-        for label, threads in (("all_cores", host_cores), ("one_core", 1)):
+        for label, threads in modes:
+            threads = threads or host_cores
             orc.set_max_threads(threads)
             steps, el = _time_oracle(orc, n, K, w.k_scale, w.v_scale, secs)
             out[label] = {"tokens_per_s": round(T * steps / el, 3), "steps": steps, "seconds": round(el, 2)}
@@ -863,12 +864,12 @@ def oracle_configs_arm(args):
     del w, n
     w = wl.prefill_chunk(seed=args.seed)
     n = w.numpy()
-    if args.oracle_full_prefill:
-        res.append(time_config(w, n, w.K, "every query row (8,192), all four stages"))
-    else:
-        idx = np.unique(np.linspace(0, w.T - 1, 64).astype(int))
-        res.append(time_config(w, rows_of(n, idx), w.K,
-                               f"{idx.size} of the {w.T:,} query rows, evenly spaced, all four stages"))
+    idx = np.unique(np.linspace(0, w.T - 1, 64).astype(int))
+    res.append(time_config(w, rows_of(n, idx), w.K,
+                           f"{idx.size} of the {w.T:,} query rows, evenly spaced, all four stages"))
+    if args.oracle_full_prefill:   # once, on every core (one core would take about half an hour)
+        res.append(time_config(w, n, w.K, f"every query row ({w.T:,}), all four stages, once",
+                               modes=(("all_cores", None),)))
     del w, n
     for case in wl.SWEEP_CASES:
         ctx, B, heads, K, kv, dist = case
@@ -905,7 +906,7 @@ def main(argv=None):
     ap.add_argument("--oracle-configs", action="store_true",
                     help="with --impl reference: time the oracle on every config (host only)")
     ap.add_argument("--oracle-full-prefill", action="store_true",
-                    help="with --oracle-configs: every query row of the prefill chunk, not 64")
+                    help="with --oracle-configs: also every query row of the prefill chunk, once")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
