@@ -355,11 +355,34 @@ __device__ __forceinline__ int count_vs(const Keys& keys, uint32_t tau) {
 // in it; when those exact counts put the n-th key inside the window (and the
 // window holds at most kListCapG keys), the window's keys are listed with their
 // ids and four digit passes over them alone find tau (the window bin, then
-// bits 12..19, 4..11 and 0..3).  Returns false, with nothing written, when the
-// guess fails; the caller then runs the radix passes.  (Block-uniform.)
+// bits 12..19, 4..11 and 0..3).  The output then needs no pass over the keys:
+// the masks of keys above and in the window, with the list, say which are kept.
+// Returns false, with nothing written, when the guess fails; the caller then
+// runs the radix passes.  (Block-uniform.)
+struct RowGuess {
+  uint32_t tau;        // the key of the n-th largest candidate
+  int need;            // keys equal to tau that are kept (the lowest ids first)
+  uint64_t above;      // this thread's keys above the window (all kept)
+  uint64_t cand;       // this thread's keys in the window
+  int pos0;            // where this thread's window keys start in the list
+};
+
+// A thread's window keys, read back from the window list (key j of the
+// thread is list entry pos0 + the number of window keys before it).
+struct ListKeys {
+  static constexpr int kUnroll = 1;
+  const uint2* list;
+  int pos0;
+  uint64_t cand;
+  __device__ __forceinline__ uint32_t get(int j) const {
+    return list[pos0 + __popcll((long long)(cand & ((1ull << j) - 1ull)))].x;
+  }
+};
+
 template <int KPT>
-__device__ __forceinline__ bool row_guess(TopkSmemG& sm, const RegKeys<KPT>& keys, int first, int c, int n,
-                                          uint32_t& tau, int& need) {
+__device__ __forceinline__ bool row_guess(TopkSmemG& sm, const RegKeys<KPT>& keys, const float* row, int first,
+                                          int c, int n, RowGuess& g) {
+  static_assert(KPT <= 64, "key masks are 64 bits");
   static_assert(KPT % 4 == 0 && kThreads * 8 == kPrefixBins, "4 samples per thread, 8 bins per thread");
   constexpr int SS = KPT / 4;  // sample stride
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -397,25 +420,28 @@ __device__ __forceinline__ bool row_guess(TopkSmemG& sm, const RegKeys<KPT>& key
   const uint32_t pb = (uint32_t)sm.pbin, pb_lo = (uint32_t)sm.pbin_lo;
   if (pb - pb_lo >= (uint32_t)kBins) return false;  // the window does not fit one 256-bin pass
 
-  // ---- verify: exact counts above the window and in it
-  int mine = 0, above = 0;
+  // ---- verify: exact counts above the window and in it (and which keys)
+  uint64_t am = 0, cm = 0;
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
     const uint32_t b = keys.get(j) >> kPrefixShift;
     const bool valid = first + j < c;
-    above += valid && b > pb;
-    mine += valid && b <= pb && b >= pb_lo;
+    if (valid && b > pb) am |= 1ull << j;
+    if (valid && b <= pb && b >= pb_lo) cm |= 1ull << j;
   }
   int tot;  // candidates (low 16 bits; c <= 32,768) and keys above the window (high)
-  int pos = block_exclusive_scan(mine | (above << 16), sm.wa, tot) & 0xffff;
+  int pos = block_exclusive_scan(__popcll((long long)cm) | (__popcll((long long)am) << 16), sm.wa, tot) & 0xffff;
   const int in_win = tot & 0xffff, above_all = tot >> 16;
   if (!(above_all < n && above_all + in_win >= n && in_win <= kListCapG)) return false;
+  g.above = am;
+  g.cand = cm;
+  g.pos0 = pos;
 
-  // ---- refine: the window's keys with their ids, in id order
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) {
-    const uint32_t k = keys.get(j), b = k >> kPrefixShift;
-    if (first + j < c && b <= pb && b >= pb_lo) sm.cand[pos++] = make_uint2(k, (uint32_t)(first + j));
+  // ---- refine: the window's keys with their ids, in id order (each key read
+  // again from the row, an L1 hit, so that the loop indexes no register array)
+  for (uint64_t m = cm; m; m &= m - 1) {
+    const int j = __ffsll((long long)m) - 1;
+    sm.cand[pos++] = make_uint2(order_key(__ldg(row + first + j)), (uint32_t)(first + j));
   }
   __syncthreads();
   uint32_t pre = 0;
@@ -446,8 +472,8 @@ __device__ __forceinline__ bool row_guess(TopkSmemG& sm, const RegKeys<KPT>& key
     pre |= pass == 0 ? (pb_lo + d) << kPrefixShift : d << shift;
     nd -= sm.above[pass];
   }
-  tau = pre;
-  need = nd;
+  g.tau = pre;
+  g.need = nd;
   return true;
 }
 
@@ -469,40 +495,60 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
   }
   if (r.hrow) zero_hist_share<1>(r.hrow, 0);  // (not read by this kernel)
   const int first = tid * KPT;
+  const float* const row = a.scores + (size_t)t * a.score_stride;
   RegKeys<KPT> keys;
-  load_keys<KPT>(keys, a.scores + (size_t)t * a.score_stride, first, r.c, vec);
+  load_keys<KPT>(keys, row, first, r.c, vec);
   // (dependents launch when this grid completes: launched earlier, their CTAs
   // compete for the SMs this kernel still needs)
 
+  if constexpr (GVR) {
+    RowGuess g;
+    if (row_guess<KPT>(sm, keys, row, first, r.c, r.n, g)) {
+      // kept: the keys above the window, then the window's keys > tau and the
+      // first g.need == tau by id (this thread's are list entries pos0 ..)
+      int gt = __popcll((long long)g.above), eq = 0;
+      const int end = g.pos0 + __popcll((long long)g.cand);
+      for (int i = g.pos0; i < end; ++i) {
+        const uint32_t k = sm.cand[i].x;
+        gt += k > g.tau;
+        eq += k == g.tau;
+      }
+      int both;
+      const int before = block_exclusive_scan(gt | (eq << 16), sm.wa, both);
+      const ListKeys lk{sm.cand, g.pos0, g.cand};
+      emit_kept<KPT, true>(sm, lk, g.above, g.cand, first, g.tau, gt, before & 0xffff, before >> 16,
+                           both & 0xffff, both >> 16, g.need, 0, r, tvec);
+      write_tail(a, r, t);
+      if (tid == 0 && a.path) a.path[t] = 1;
+      return;
+    }
+  }
+
+  // ---- radix select: four passes of 8 bits from the top
   uint32_t prefix = 0;
   int need = r.n;  // how many keys matching `prefix` are still to be taken
-  bool guessed = false;
-  if constexpr (GVR) guessed = row_guess<KPT>(sm, keys, first, r.c, r.n, prefix, need);
-  // ---- radix select: four passes of 8 bits from the top
-  if (!guessed) {
 #pragma unroll
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
 #pragma unroll
-      for (int b = threadIdx.x & 31; b < kBins; b += 32) sm.hw[warp][b] = 0u;
-      __syncwarp();
+    for (int b = threadIdx.x & 31; b < kBins; b += 32) sm.hw[warp][b] = 0u;
+    __syncwarp();
 #pragma unroll
-      for (int j = 0; j < KPT; ++j) {
-        const uint32_t k = keys.get(j);
-        const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
-        if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
-      }
-      __syncthreads();
-      if (tid < kBins) {
-        uint32_t v = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
-        find_bin((int)v, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
-      }
-      __syncthreads();
-      prefix |= (uint32_t)sm.bin[pass] << shift;
-      need -= sm.above[pass];
+    for (int j = 0; j < KPT; ++j) {
+      const uint32_t k = keys.get(j);
+      const bool match = pass == 0 ? k != 0u : (k >> (shift + 8)) == (prefix >> (shift + 8));
+      if (match) atomicAdd(&sm.hw[warp][(k >> shift) & (kBins - 1)], 1u);
     }
+    __syncthreads();
+    if (tid < kBins) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) v += sm.hw[w][kBins - 1 - tid];
+      find_bin((int)v, need, kBins - 1 - tid, &sm.bin[pass], &sm.above[pass], sm.wa);
+    }
+    __syncthreads();
+    prefix |= (uint32_t)sm.bin[pass] << shift;
+    need -= sm.above[pass];
   }
   const uint32_t tau = prefix;
 
@@ -513,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 2) topk_row_kernel(TopkArgs a, int v
   emit_kept<KPT, false>(sm, keys, 0, 0, first, tau, ge & 0xffff, before & 0xffff, before >> 16, both & 0xffff,
                         both >> 16, need, 0, r, tvec);
   write_tail(a, r, t);
-  if (GVR && tid == 0 && a.path) a.path[t] = guessed ? 1 : 3;
+  if (GVR && tid == 0 && a.path) a.path[t] = 3;
 }
 
 // ---- few long rows: one cluster per row, keys in shared memory ------------------
