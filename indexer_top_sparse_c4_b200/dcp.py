@@ -19,7 +19,7 @@ the stacked per-shard buffers.
 """
 from __future__ import annotations
 
-from typing import List, Optional, Tuple
+from typing import List, Tuple
 
 import torch
 

@@ -4,7 +4,6 @@ selection: out, lse and the status bits bit for bit.  The gather kernel's
 own token listing (few rows), and the expand-into-workspace fallback of the
 other plans (many rows on the streaming kernel; FP32 caches on the general
 kernel); bad group ids and rows wider than W."""
-import numpy as np
 import pytest
 import torch
 
